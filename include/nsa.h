@@ -258,8 +258,12 @@ size_t nsa_workspace_bytes(int B, int Hq, int Hkv, int Sq, int Skv, int D,
  *  - Sizes whose workspace (nsa_workspace_bytes) exceeds the array are
  *    rejected with NSA_ERR_INVALID_ARG and a message naming the limit.
  *  - The first call on a device looks up the array's device address with
- *    cudaGetSymbolAddress (with that device current); make that first call
- *    before any stream capture.
+ *    cudaGetSymbolAddress (with that device current). With lazy module
+ *    loading (the CUDA default) that lookup may load the library's device
+ *    code on that device, which is when the array is reserved, and it may
+ *    synchronise. Make one warm-up call on each device at initialisation
+ *    (or set CUDA_MODULE_LOADING=EAGER), and in any case before any stream
+ *    capture.
  *  - All calls share the array: calls whose work overlaps on the GPU (on
  *    different streams, or from different threads) race. The array keeps the
  *    last call's contents; nothing in it needs to start at zero. */
@@ -349,8 +353,29 @@ nsa_status nsa_radial_blocks(int B, int Sq, int Skv, double density,
 
 /* Reads (and with clear != 0 resets) the library's device error word on the
  * current device, synchronising the device first. Returns NSA_ERR_TIMEOUT if
- * a kernel's bounded wait gave up since the last clear, else NSA_OK. */
+ * a kernel's bounded wait gave up since the last clear, else NSA_OK; the
+ * message then names the wait site code of the first wait that gave up. */
 nsa_status nsa_device_status(int clear);
+
+/* Failure detection check (no counterpart on the pages): every wait inside
+ * the library's kernels is bounded (about one second of SM clock), and a wait
+ * that runs out records NSA_ERR_TIMEOUT and its site code in the device error
+ * word, drains what its CTA has in flight and returns, leaving the context
+ * usable. This call enqueues a one-CTA kernel whose single wait, with a limit
+ * of limit_cycles SM clock cycles (1 .. the kernels' own limit), is on a
+ * condition nothing satisfies: which = 0 waits on an mbarrier no thread
+ * arrives on (site 0x70), which = 1 on a counter no thread increments (site
+ * 0x71). The kernel has nothing in flight while it waits. After it,
+ * nsa_device_status reports NSA_ERR_TIMEOUT with that site; later calls run
+ * normally. NSA_ERR_INVALID_ARG for other values of which or limit_cycles. */
+nsa_status nsa_selftest_timeout(int which, long long limit_cycles,
+                                nsa_stream_t stream);
+
+/* Number of kernels the library has launched in this process so far, over
+ * every device and host thread (memsets and copies are not counted). Host
+ * only, no CUDA call. The difference of two readings counts the kernels a
+ * span of calls launched. */
+unsigned long long nsa_kernel_launches(void);
 
 #ifdef __cplusplus
 }

@@ -187,3 +187,43 @@ def test_wrappers_with_a_stream_allocate_on_it():
                 assert getattr(f, "__wrapped__", None) is not None, name
                 seen.append(name)
     assert "nsa_forward" in seen and "nsa_block_sparse_attn_bwd" in seen and len(seen) >= 10
+
+
+def test_stream_given_by_position_is_entered(monkeypatch):
+    # a stream passed positionally must be entered like one passed by keyword,
+    # or the wrapper's allocations would land on the current stream instead
+    from top_kv_tile_b200 import binding
+    entered = []
+
+    class Ctx:
+        def __init__(self, s):
+            self.s = s
+
+        def __enter__(self):
+            entered.append(self.s)
+
+        def __exit__(self, *exc):
+            return False
+
+    monkeypatch.setattr(binding.torch.cuda, "stream", Ctx)
+
+    @binding._on_caller_stream
+    def f(x, block, out=None, stream=None):
+        return stream
+
+    s = object()
+    assert f(1, 2, None, s) is s and entered == [s]
+    assert f(1, 2, stream=s) is s and entered == [s, s]
+    assert f(1, 2) is None and entered == [s, s]
+
+
+def test_selftest_timeout_and_launch_count_on_host(nsa):
+    L = nsa.lib()
+    # invalid arguments are rejected before any CUDA call
+    assert L.nsa_selftest_timeout(2, 1000, None) == nsa.NSA_ERR_INVALID_ARG
+    assert L.nsa_selftest_timeout(0, 0, None) == nsa.NSA_ERR_INVALID_ARG
+    assert L.nsa_selftest_timeout(1, 1 << 40, None) == nsa.NSA_ERR_INVALID_ARG
+    assert "limit_cycles" in nsa.nsa_last_error()
+    # the launch counter is a plain host read
+    n = nsa.nsa_kernel_launches()
+    assert isinstance(n, int) and n >= 0 and nsa.nsa_kernel_launches() == n

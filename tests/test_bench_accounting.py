@@ -36,14 +36,19 @@ def test_kept_tile_flops_per_query_head():
     assert bench.kept_tile_flops(shared, wl) == 5 * wl.Hq * per_tile
 
 
-def test_launches_per_step_by_path():
-    # gqa: 128 kv tiles * 128 dims * 4 B = 64 KB of pooled keys per head
-    #   (resident) and 8 * 16 * 2 = 256 select CTAs <= 2 per SM * 148: one
-    #   cooperative select kernel + attention = 2
-    # cross: 250 * 64 * 4 B < 64 KB, 4 * 8 * 4 = 128 CTAs: 2
-    # large2d: 2048 * 128 * 4 B = 1 MB, not resident, 2048 tiles <= 2048:
-    #   pool + tensor-core scores + top-k from scores + attention = 4
-    # head_shared: pool + 2 head means + tensor-core scores + top-k + attention = 6
-    expect = {"gqa": 2, "cross": 2, "large2d": 4, "head_shared": 6}
-    for name, n in expect.items():
-        assert bench.launches_per_step(workloads.get(name)) == n, name
+def test_plan_kept_flops_by_hand():
+    # tiny: 8 query tiles x 16 kv tiles, 2 diagonal tiles per row, 14
+    # candidates, ceil(14 * 0.3) = 5, so 7 kept per row; 2 heads; D = 64
+    wl = workloads.get("tiny")
+    assert bench.plan_kept_flops(wl, None, None) == 7 * 8 * 2 * 4 * 128 * 64 * 64
+    # head_shared: 53 kept per row of 256, one keep head for 32 query heads
+    wl = workloads.get("head_shared")
+    assert bench.plan_kept_flops(wl, None, None) == 53 * 256 * 32 * 4 * 128 * 64 * 128
+    # gqa: 40 kept per row, 64 rows, 2 batches, 16 heads
+    wl = workloads.get("gqa")
+    assert bench.plan_kept_flops(wl, None, None) == 40 * 64 * 2 * 16 * 4 * 128 * 64 * 128
+
+
+def test_oracle_units_cover_each_kv_group_once():
+    assert bench.oracle_units(workloads.get("gqa")) == [(b, hk) for b in range(2) for hk in range(4)]
+    assert bench.oracle_units(workloads.get("head_shared")) == [(0, None)]

@@ -77,10 +77,18 @@ def _same(a, b):
 
 
 def test_noalloc_matches_workspace_path_on_consecutive_calls(nsa):
-    cases = [_inputs("gqa_small"), _inputs("cross_small")]
+    # the paths a call can take: the single cooperative select kernel
+    # (gqa_small, cross_small), pooling first with the head means
+    # (head_shared_small), tensor-core scores for long rows (long_kv_hs) and
+    # a partial last tile on both axes (ragged)
+    names = ["gqa_small", "cross_small", "head_shared_small", "long_kv_hs", "ragged"]
+    cases = [_inputs(n) for n in names]
+    for wl, _ in cases:
+        spec = nsa.SparseSpec(wl.budget, wl.block_q, wl.block_kv, wl.head_shared, wl.force)
+        assert nsa.nsa_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.Sq, wl.Skv, wl.D, spec) <= nsa.NOALLOC_SCRATCH_BYTES
     refs = [_with_workspace(nsa, wl, d) for wl, d in cases]
-    # two calls in a row per case, interleaved so each call finds the other
-    # case's leftovers in the shared scratch array
+    # two calls in a row per case, interleaved so each call finds another
+    # path's leftovers in the shared scratch array
     for _ in range(2):
         for (wl, d), ref in zip(cases, refs):
             _same(_noalloc_c_abi(nsa, wl, d), ref)

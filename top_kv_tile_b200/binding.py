@@ -12,6 +12,7 @@ from __future__ import annotations
 
 import ctypes
 import functools
+import inspect
 import math
 import os
 from dataclasses import dataclass
@@ -36,7 +37,8 @@ SYMBOLS = ("nsa_last_error", "nsa_version", "nsa_pool", "nsa_score", "nsa_select
            "nsa_workspace_bytes", "nsa_device_status", "nsa_forward_noalloc", "nsa_plan_bytes",
            "nsa_plan_build", "nsa_forward_plan", "nsa_schedule", "nsa_radial_blocks",
            "nsa_block_sparse_attn_fwd_masked", "nsa_block_sparse_attn_bwd", "nsa_bwd_workspace_bytes",
-           "nsa_block_sparse_attn_bwd_masked", "nsa_score_tc")
+           "nsa_block_sparse_attn_bwd_masked", "nsa_score_tc", "nsa_selftest_timeout",
+           "nsa_kernel_launches")
 
 
 class NsaError(RuntimeError):
@@ -114,6 +116,10 @@ _lib.nsa_workspace_bytes.restype = _SZ
 _lib.nsa_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I, _PSPEC]
 _lib.nsa_device_status.restype = _I
 _lib.nsa_device_status.argtypes = [_I]
+_lib.nsa_selftest_timeout.restype = _I
+_lib.nsa_selftest_timeout.argtypes = [_I, ctypes.c_longlong, _P]
+_lib.nsa_kernel_launches.restype = ctypes.c_ulonglong
+_lib.nsa_kernel_launches.argtypes = []
 
 
 class nsa_plan_info(ctypes.Structure):
@@ -158,16 +164,20 @@ def _ptr(t):
 
 
 def _on_caller_stream(fn):
-    """Runs a wrapper under its caller's `stream` (when one is given), so that
-    the tensors it allocates (workspace, converted masks, outputs) belong to
-    the stream its kernels run on and the caching allocator does not hand
-    their memory to another stream while those kernels may still use it."""
+    """Runs a wrapper under its caller's `stream` (when one is given, by
+    keyword or by position), so that the tensors it allocates (workspace,
+    converted masks, outputs) belong to the stream its kernels run on and the
+    caching allocator does not hand their memory to another stream while
+    those kernels may still use it."""
+    sig = inspect.signature(fn)
+
     @functools.wraps(fn)
-    def wrapper(*args, stream=None, **kwargs):
+    def wrapper(*args, **kwargs):
+        stream = sig.bind(*args, **kwargs).arguments.get("stream")
         if stream is None:
             return fn(*args, **kwargs)
         with torch.cuda.stream(stream):
-            return fn(*args, stream=stream, **kwargs)
+            return fn(*args, **kwargs)
     return wrapper
 
 
@@ -465,6 +475,19 @@ def nsa_forward(q, k, v, spec: SparseSpec, scale: float | None = None, pins=None
 def nsa_device_status(clear: bool = True) -> None:
     """Raises NsaError(TIMEOUT) if a kernel's bounded wait gave up."""
     _check(_lib.nsa_device_status(int(clear)))
+
+
+@_on_caller_stream
+def nsa_selftest_timeout(which: int, limit_cycles: int, stream=None) -> None:
+    """Enqueues the kernel whose one bounded wait runs out (which 0: an
+    mbarrier, site 0x70; 1: a counter, site 0x71) after limit_cycles SM
+    cycles; nsa_device_status() then raises NsaError(TIMEOUT)."""
+    _check(_lib.nsa_selftest_timeout(int(which), int(limit_cycles), _stream(stream)))
+
+
+def nsa_kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(_lib.nsa_kernel_launches())
 
 
 NOALLOC_SCRATCH_BYTES = 16 << 20

@@ -810,6 +810,7 @@ cudaError_t launch_bwd_t(const AttnBwdArgs &a, const __nv_bfloat16 *out, const _
     long long blocks = (rows * (D / 8) + 255) / 256;
     if (blocks > (long long)num_sms * 16) blocks = (long long)num_sms * 16;
     bwd_dvec_kernel<D><<<(int)blocks, 256, 0, stream>>>(out, dout, rows, a.dvec);
+    note_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // per kv tile the query tiles that kept it
@@ -821,6 +822,7 @@ cudaError_t launch_bwd_t(const AttnBwdArgs &a, const __nv_bfloat16 *out, const _
       keep_to_qindex_kernel<<<(int)blocks, 256, 0, stream>>>(keep, (long long)a.B * a.Hs, a.NQ, a.NK,
                                                             const_cast<int32_t *>(a.q_count),
                                                             const_cast<uint16_t *>(a.q_index));
+      note_launch();
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
   }

@@ -3,6 +3,7 @@
 // point allocates device or pinned memory; all buffers belong to the caller.
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -10,6 +11,7 @@
 #include <string>
 
 #include "../../include/nsa.h"
+#include "nsa_device.cuh"
 #include "nsa_kernels.cuh"
 
 namespace {
@@ -304,9 +306,13 @@ nsa::SelectArgs select_args(const float *pq, const float *pk, const Geometry &g,
   return a;
 }
 
+std::atomic<unsigned long long> g_launches{0};
+
 }  // namespace
 
 void nsa::set_last_error(const char *msg) { g_last_error = msg; }
+
+void nsa::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 extern "C" {
 
@@ -732,6 +738,21 @@ nsa_status nsa_block_sparse_attn_bwd_masked(const void *q, const void *k, const 
   }
   NSA_CUDA(nsa::launch_attn_bwd(a, D, static_cast<const __nv_bfloat16 *>(out),
                                 static_cast<const __nv_bfloat16 *>(dout), keep, dev->num_sms, tq, tdo, tk, tv, s));
+  return NSA_OK;
+}
+
+unsigned long long nsa_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+nsa_status nsa_selftest_timeout(int which, long long limit_cycles, nsa_stream_t stream) {
+  g_last_error.clear();
+  if (which != 0 && which != 1) return fail(NSA_ERR_INVALID_ARG, "nsa_selftest_timeout: which must be 0 or 1");
+  if (limit_cycles < 1 || limit_cycles > nsa::kWaitLimitCycles)
+    return fail(NSA_ERR_INVALID_ARG, "nsa_selftest_timeout: limit_cycles must be in [1, %lld]",
+                nsa::kWaitLimitCycles);
+  DeviceInfo *dev;
+  nsa_status st = device_info(&dev);
+  if (st != NSA_OK) return st;
+  NSA_CUDA(nsa::launch_selftest_wait(which, limit_cycles, dev->err, (cudaStream_t)stream));
   return NSA_OK;
 }
 

@@ -85,26 +85,53 @@ __device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t pa
   return ok != 0;
 }
 
+// Records a timed-out wait in the device error word: the timeout bit, and
+// the site code unless an earlier wait already left one.
+__device__ __forceinline__ void note_timeout(unsigned int *err, unsigned int site) {
+  atomicOr(err, kErrTimeout);
+  atomicCAS(err + 1, 0u, site);
+}
+
 // Waits for the phase with the given parity to complete. Gives up after
-// kWaitLimitCycles or as soon as *abort is set by another role of the CTA;
-// on a timeout it records the error in *err and sets *abort. Returns false
-// when the caller must stop. The waiting thread sleeps in the barrier
-// (suspended try_wait) rather than spinning, so that it leaves the issue
-// slots of its SM sub-partition to the warps that compute.
+// `limit` SM clock cycles (kWaitLimitCycles unless a caller passes less) or
+// as soon as *abort is set by another role of the CTA; on a timeout it
+// records the error in *err and sets *abort. Returns false when the caller
+// must stop. The waiting thread sleeps in the barrier (suspended try_wait)
+// rather than spinning, so that it leaves the issue slots of its SM
+// sub-partition to the warps that compute.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          unsigned int *err, unsigned int site = 0xFFu) {
+                                          unsigned int *err, unsigned int site = 0xFFu,
+                                          long long limit = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = clock64();
   while (true) {
     if (mbar_try_wait_suspend(bar, parity, 200000u)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       *abort = 1;
-      atomicOr(err, kErrTimeout);
-      atomicCAS(err + 1, 0u, site);
+      note_timeout(err, site);
       return false;
     }
   }
+}
+
+// Waits until the counter *ctr (global or shared memory, written by other
+// CTAs or threads with atomics) reaches `target`, sleeping briefly between
+// reads. Gives up after `limit` SM clock cycles, recording the timeout and
+// `site` in *err; returns false then. A fence after a successful wait orders
+// the caller's later reads after the writes the counter announced.
+__device__ __forceinline__ bool counter_wait(unsigned int *ctr, unsigned int target, unsigned int *err,
+                                             unsigned int site, long long limit = kWaitLimitCycles) {
+  const long long t0 = clock64();
+  while (atomicAdd(ctr, 0u) < target) {
+    if (clock64() - t0 > limit) {
+      note_timeout(err, site);
+      return false;
+    }
+    __nanosleep(128);
+  }
+  __threadfence();
+  return true;
 }
 
 // ----------------------------------------------------------------------- TMA

@@ -10,6 +10,9 @@
 
 namespace nsa {
 
+// Counts one kernel launched by the library (nsa_kernel_launches()).
+void note_launch();
+
 // Launches `kernel` on `stream` with programmatic stream serialization, so it
 // can be scheduled while the previous kernel on the stream drains; the kernel
 // calls pdl_wait() before touching its predecessor's outputs.
@@ -26,7 +29,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e == cudaSuccess) note_launch();
+  return e;
 }
 
 // One tensor to pool: x (BH, S, D) bf16 -> out (BH, ntiles, D) f32.
@@ -203,6 +208,11 @@ cudaError_t launch_attn_bwd(const AttnBwdArgs &a, int D, const __nv_bfloat16 *ou
                             const CUtensorMap &tk, const CUtensorMap &tv, cudaStream_t stream);
 
 
+
+// A one-CTA kernel whose single bounded wait (which 0: an mbarrier, site
+// 0x70; which 1: a counter, site 0x71) runs out after limit_cycles and
+// records the timeout in err (selftest.cu).
+cudaError_t launch_selftest_wait(int which, long long limit_cycles, unsigned int *err, cudaStream_t stream);
 
 // Sets the calling thread's nsa_last_error() message.
 void set_last_error(const char *msg);

@@ -14,8 +14,11 @@
 // every GPU on which the library's kernels are loaded holds it until the
 // process exits. Host code cannot use the array's name as a device address,
 // so the first call on each device looks the address up with
-// cudaGetSymbolAddress (with that device current) and caches it; that first
-// call should be made before any stream capture. Every call shares the one
+// cudaGetSymbolAddress (with that device current) and caches it. Under lazy
+// module loading (the CUDA default) that lookup may load the library's
+// device code on the device, reserving the array then, and may synchronise:
+// callers should make one warm-up call per device at initialisation (or run
+// with CUDA_MODULE_LOADING=EAGER), and in any case before any stream capture. Every call shares the one
 // array: two calls whose work overlaps on the GPU (e.g. on two streams) race
 // and give wrong results. Nothing in the array needs to start at zero: the
 // pooling kernel clears the plan flag and every other scratch byte a call

@@ -163,11 +163,13 @@ cudaError_t launch_plan_build(const PlanArgs &p, int num_sms, cudaStream_t strea
   long long blocks = (rows + 7) / 8;
   if (blocks > (long long)num_sms * 8) blocks = (long long)num_sms * 8;
   plan_build_kernel<<<(int)blocks, 256, 0, stream>>>(p);
+  note_launch();
   return cudaGetLastError();
 }
 
 cudaError_t launch_radial(const RadialArgs &r, int num_sms, cudaStream_t stream) {
   radial_width_kernel<<<1, kRadialThreads, 0, stream>>>(r);
+  note_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const long long rows = (long long)r.B * r.NQ;
@@ -175,6 +177,7 @@ cudaError_t launch_radial(const RadialArgs &r, int num_sms, cudaStream_t stream)
   long long blocks = (rows + 7) / 8;
   if (blocks > (long long)num_sms * 8) blocks = (long long)num_sms * 8;
   radial_write_kernel<<<(int)blocks, 256, 0, stream>>>(r);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -201,6 +201,7 @@ cudaError_t launch_pool_d(const PoolSeg &a, const PoolSeg &b, int grid, unsigned
   cudaError_t e = cudaFuncSetAttribute(pool_kernel<D, W>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   pool_kernel<D, W><<<grid, W * 32, smem, stream>>>(a, b, clear_word, err);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -772,23 +772,13 @@ __global__ void __launch_bounds__(kThreads) select_fusedq_kernel(SelectArgs a) {
   if (a.k_raw != nullptr) {
     // the warps that found the group incomplete: wait for it (bounded)
     if (!__syncthreads_and(issued)) {
-      if (tid == 0) {
-        int stop = 0;
-        const long long t_start = clock64();
-        while (atomicAdd(ctr, 0u) < (unsigned int)n_group) {
-          if (clock64() - t_start > kWaitLimitCycles) {
-            atomicOr(a.err, kErrTimeout);
-            atomicCAS(a.err + 1, 0u, 0x30u);
-            stop = 1;
-            break;
-          }
-          __nanosleep(128);
-        }
-        __threadfence();  // the group's pooled rows after the count
-        s_stop = stop;
-      }
+      // (the fence in counter_wait orders the group's pooled rows after the count)
+      if (tid == 0) s_stop = counter_wait(ctr, (unsigned int)n_group, a.err, 0x30u) ? 0 : 1;
       __syncthreads();
-      if (s_stop) return;
+      if (s_stop) {
+        cp_async_wait<0>();  // key copies a warp issued early land before the CTA exits
+        return;
+      }
       if (!issued) load_keys();
     }
   } else {
@@ -996,7 +986,9 @@ cudaError_t launch_coop(K kernel, dim3 grid, size_t smem, const SelectArgs &a, c
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, a);
+  e = cudaLaunchKernelEx(&cfg, kernel, a);
+  if (e == cudaSuccess) note_launch();
+  return e;
 }
 
 template <typename K>
@@ -1102,6 +1094,7 @@ cudaError_t launch_keep_to_index(const int8_t *keep, long long rows, int NK, int
   long long blocks = (rows + 7) / 8;
   if (blocks > 148LL * 16) blocks = 148LL * 16;
   keep_to_index_kernel<<<(int)blocks, 256, 0, stream>>>(keep, rows, NK, kv_count, kv_index);
+  note_launch();
   return cudaGetLastError();
 }
 

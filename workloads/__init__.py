@@ -130,6 +130,13 @@ _W += [
              budget=0.15, pins_drops="sinks2_blockcausal"),
     Workload("long_kv_hs", B=1, Hq=4, Hkv=2, Sq=512, Skv=16384, D=128,
              budget=0.10, head_shared=True),
+    # one kv group of the Large 2D-local workload (8 query heads, 1/8 of its
+    # work), for profiling captures that must stay small; per kv group the
+    # kernels see the same shapes, statistics and schedule
+    Workload("large2d_1kv", B=1, Hq=8, Hkv=1, Sq=131072, Skv=131072, D=128,
+             budget=0.05, recipe="fourier2d",
+             params={"rows": 256, "cols": 512, "modes": 16, "fmax": 1.0 / 32,
+                     "noise": 0.3}),
 ]
 
 WORKLOADS = {w.name: w for w in _W}
