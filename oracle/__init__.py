@@ -17,7 +17,7 @@ is "parity unpinned".
 """
 from .selector import (  # noqa: F401
     SparseSpec, block_count, pool_blocks, diagonal_blocks, head_map,
-    score_blocks, selection_plan, select_blocks, keep_to_lists,
+    score_blocks, selection_plan, select_blocks, select_pooled, keep_to_lists,
     boundary_scores, radial_blocks, schedule, budget_count, select_rows,
 )
 from .attention import block_sparse_attention, attention_tiles, block_sparse_attention_bwd  # noqa: F401

@@ -144,15 +144,27 @@ def select_blocks(q, k, spec: SparseSpec, pins=None, drops=None, return_scores=F
     descending sort); a candidate is kept when its rank is below the row's
     budget count; must tiles are added and forbidden tiles removed last.
     With ``return_scores`` the float64 scores and the plan come back as well.
+    The pooling step is ``pool_blocks``; the rest is ``select_pooled``.
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
-    nq = block_count(q.shape[-2], spec.block_q)
-    nk = block_count(k.shape[-2], spec.block_kv)
+    return select_pooled(pool_blocks(q, spec.block_q), pool_blocks(k, spec.block_kv), spec, pins, drops,
+                         return_scores)
+
+
+def select_pooled(pq, pk, spec: SparseSpec, pins=None, drops=None, return_scores=False):
+    """``select_blocks`` from the pooled tensors on: pq (B, Hq, NQ, D) and pk
+    (B, Hkv, NK, D) as ``pool_blocks`` gives them. The head handling of
+    ``score_blocks`` (``head_map``), the unscaled scores, the plan and the
+    ranking, with the same results and return values as ``select_blocks``."""
+    pq = np.asarray(pq, dtype=np.float64)
+    pk = np.asarray(pk, dtype=np.float64)
+    nq, nk = pq.shape[-2], pk.shape[-2]
     must, forbidden, cand, kpr, covers = selection_plan(spec, nq, nk, pins, drops)
     if covers and not spec.force:
         return (None, None, None) if return_scores else None
-    scores = score_blocks(q, k, spec)
+    hq, hk = head_map(pq, pk, spec.head_shared)
+    scores = np.matmul(hq, np.swapaxes(hk, -1, -2))
     shape = scores.shape
     cand_b = np.broadcast_to(cand, shape)
     masked = np.where(cand_b, scores, -np.inf)

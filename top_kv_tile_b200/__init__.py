@@ -15,7 +15,7 @@ import importlib
 
 # submodules that must import without libnsa.so (``from top_kv_tile_b200
 # import build`` asks the package for the attribute before the submodule)
-_SUBMODULES = ("build", "binding")
+_SUBMODULES = ("build", "binding", "shard")
 
 
 def __getattr__(name):
