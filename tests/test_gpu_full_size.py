@@ -2,9 +2,9 @@
 bench.py times (nsa_forward with keep_out).
 
 Keep rows: Tiny, GQA and Cross are checked row by row against the oracle's
-full select_blocks; Head-shared and Large2D (too large for the oracle to
-select in full within a test) against oracle.select_rows on 256 sampled rows
-plus the corner rows. Every row of every workload also satisfies properties
+full select_blocks; Head-shared (all 256 rows) and Large2D (256 sampled rows
+plus the corner rows; too large for the oracle to select in full within a
+test) against oracle.select_rows. Every row of every workload also satisfies properties
 that hold at any size: kept count = |must \\ forbidden| + ceil(c * budget) and
 every must-and-not-forbidden tile present.
 
@@ -104,8 +104,11 @@ def test_full_size_from_the_oracle_keep(nsa, name):
         stats = parity.check_keep_rows(gk, okeep, scores, plan)
         oracle_row = {r: okeep[r] for r in map(keep_row_of, tiles)}
     else:
-        rows = {(int(rng.integers(wl.B)), int(rng.integers(wl.Hs)), int(rng.integers(wl.NQ)))
-                for _ in range(N_KEEP_ROWS)}
+        if wl.B * wl.Hs * wl.NQ <= 2 * N_KEEP_ROWS:
+            rows = set(np.ndindex(wl.B, wl.Hs, wl.NQ))  # head_shared: all 256 rows
+        else:
+            rows = {(int(rng.integers(wl.B)), int(rng.integers(wl.Hs)), int(rng.integers(wl.NQ)))
+                    for _ in range(N_KEEP_ROWS)}
         rows |= {(0, 0, 0), (wl.B - 1, wl.Hs - 1, wl.NQ - 1)}
         rows |= set(map(keep_row_of, tiles))
         rows = sorted(rows)

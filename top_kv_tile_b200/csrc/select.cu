@@ -29,7 +29,7 @@
 //     float -> larger key, -0 == +0, every finite candidate key >= 1, non
 //     candidates 0). One warp per row finds the k-th largest key T (rows
 //     of up to 256 tiles: a bitonic sort of the keys across the warp;
-//     longer rows: radix selection, four 8-bit digit passes), then keeps every
+//     longer rows: repeated 256-bin bucketing of the keys' range), then keeps every
 //     key > T and the lowest-index keys == T up to k: exactly the stable
 //     descending argsort's first k, ties to the lower kv index. Rows of up to 2048 tiles keep
 //     their keys in registers; longer rows keep them in shared memory.
@@ -173,20 +173,37 @@ __device__ __forceinline__ uint32_t warp_kth_largest(uint32_t (&x)[N], int k) {
   return __shfl_sync(0xffffffffu, v, pos / N);
 }
 
-// The k-th largest (1 <= k <= 128 G) of the 128 G keys a warp holds (4 G per
-// lane), by radix selection on 8-bit digits from the top: per pass a 256-bin
-// histogram (in the warp's slice of shared memory) of the keys that match
-// the digits found so far, then the digit whose bin holds the k-th largest
-// of them. Four passes give the exact key. Every lane returns the same value.
+// The k-th largest (1 <= k <= number of nonzero keys) of the nonzero keys a
+// warp holds (4 G per lane; a key of 0 marks a tile that is not a candidate).
+// Each pass divides the current key interval [lo, hi] into at most 256
+// equal-width bins, counts the keys of the interval per bin (a histogram in
+// the warp's slice of shared memory) and keeps the bin that holds the k-th
+// largest; a bin one key wide is the exact key. The first interval is the
+// keys' own range, from their minimum to their maximum: a row's scores share
+// their leading bits, so bins cut from the top bits of the key would pile
+// nearly every key into one bin (and its counter). Every lane returns the
+// same value.
 template <int G>
 __device__ __forceinline__ uint32_t warp_kth_radix(const uint32_t (&kk)[G][4], int k) {
   __shared__ int hist_all[kThreads / 32][256];
   int *hist = hist_all[threadIdx.x / 32];
   const int lane = threadIdx.x & 31;
-  uint32_t prefix = 0, pmask = 0;
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (kk[g][e] != 0u) {
+        lo = min(lo, kk[g][e]);
+        hi = max(hi, kk[g][e]);
+      }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
   int kr = k;
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  while (lo < hi) {
+    // bin width 2^shift with (hi - lo) >> shift < 256
+    const int shift = max(0, 24 - __clz(hi - lo));
     for (int q = lane; q < 256; q += 32) hist[q] = 0;
     __syncwarp();
 #pragma unroll
@@ -194,10 +211,10 @@ __device__ __forceinline__ uint32_t warp_kth_radix(const uint32_t (&kk)[G][4], i
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const uint32_t key = kk[g][e];
-        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+        if (key >= lo && key <= hi) atomicAdd(&hist[(key - lo) >> shift], 1);
       }
     __syncwarp();
-    // lane l holds digits 255 - 8 l down to 248 - 8 l (descending)
+    // lane l holds bins 255 - 8 l down to 248 - 8 l (descending)
     int c8[8], sum = 0;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -210,28 +227,30 @@ __device__ __forceinline__ uint32_t warp_kth_radix(const uint32_t (&kk)[G][4], i
       const int y = __shfl_up_sync(0xffffffffu, incl, off);
       if (lane >= off) incl += y;
     }
-    const int excl = incl - sum;  // matching keys with a larger digit than this lane's
+    const int excl = incl - sum;  // keys of the interval in higher bins than this lane's
     const bool mine = excl < kr && kr <= incl;
-    int digit = 0, above = excl;
+    int bin = 0, above = excl;
     if (mine) {
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         if (above + c8[q] >= kr) {
-          digit = 255 - (lane * 8 + q);
+          bin = 255 - (lane * 8 + q);
           break;
         }
         above += c8[q];
       }
     }
     const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
-    digit = __shfl_sync(0xffffffffu, digit, src);
+    bin = __shfl_sync(0xffffffffu, bin, src);
     above = __shfl_sync(0xffffffffu, above, src);
     kr -= above;
-    prefix |= (uint32_t)digit << shift;
-    pmask |= 0xFFu << shift;
+    const uint32_t nlo = lo + ((uint32_t)bin << shift);
+    const uint32_t width = (1u << shift) - 1u;
+    hi = (hi - nlo < width) ? hi : nlo + width;
+    lo = nlo;
     __syncwarp();  // every lane has read the histogram before it is cleared
   }
-  return prefix;
+  return lo;
 }
 
 // The row's budget count: the plan's, else ceil(f32(c) * f32(budget)).
@@ -352,15 +371,22 @@ __device__ __forceinline__ void select_rows_regs(const SelectArgs &a, const floa
         pos += __popc(kb & lt_mask);
         kept_tot += __popc(kb);
       }
+      if (krow && (NK & 3) == 0 && (reinterpret_cast<uintptr_t>(a.keep) & 3u) == 0 && jb + 3 < NK) {
+        // the lane's four keep bytes in one 4-byte store (the keep tensor is
+        // 4-byte aligned and its rows, NK bytes apart, are too)
+        *reinterpret_cast<uint32_t *>(krow + jb) =
+            (uint32_t)kp[0] | ((uint32_t)kp[1] << 8) | ((uint32_t)kp[2] << 16) | ((uint32_t)kp[3] << 24);
+      } else if (krow) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (jb + e < NK) krow[jb + e] = (int8_t)kp[e];
+      }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int j = jb + e;
-        if (j < NK) {
-          if (krow) krow[j] = (int8_t)kp[e];
-          if (kp[e]) {
-            if (irow) irow[pos] = (uint16_t)j;
-            ++pos;
-          }
+        if (j < NK && kp[e]) {
+          if (irow) irow[pos] = (uint16_t)j;
+          ++pos;
         }
       }
       tie_base += tie_tot;
