@@ -81,13 +81,15 @@ nsa_status nsa_pool(const void *x, int B, int H, int S, int D, int block,
  * scores[b,h,i,j] = <pq[b,h,i,:], pk[b,h/(Hq/Hkv),j,:]> for per-head scoring
  * (Hq % Hkv == 0), from tf32 hi/lo splits of the float32 operands with
  * hi.hi + hi.lo + lo.hi accumulated in f32 (error-compensated 3xTF32).
- * scores: f32 (B,Hq,NQ,NKP) with NKP = NK rounded up to 128; columns NK..
- * up to the next multiple of 64 are written (0), the rest of each row is
- * left untouched. D in {64,128}; pq, pk, scores 16-byte aligned. nsa_select
- * and nsa_forward use the same kernel for rows whose pooled keys exceed
- * 64 KB (NK * D * 4 > 65536) when the workspace holds the score scratch. */
+ * scores: f32 (B,Hq,NQ,NKP) with NKP = NK rounded up to 128; columns NK ..
+ * NKP-1 are written as 0. D in {64,128}; pq, pk, scores 16-byte aligned.
+ * workspace (device, 256-byte aligned, at least 2 * round_up(B*Hkv*NK*D*4,
+ * 256) bytes) receives the tf32 hi and lo parts of pk. nsa_select and
+ * nsa_forward use the same kernels for rows whose pooled keys exceed 64 KB
+ * (NK * D * 4 > 65536), in their own workspace. */
 nsa_status nsa_score_tc(const float *pq, const float *pk, int B, int Hq,
                         int Hkv, int NQ, int NK, int D, float *scores,
+                        void *workspace, size_t workspace_bytes,
                         nsa_stream_t stream);
 
 /* selector.py, score_blocks (debug/test path): unscaled pooled affinities

@@ -11,6 +11,9 @@ LSE max-abs 1e-4.
 """
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 
 import oracle
@@ -109,6 +112,11 @@ def check_grad(g, ref, name="grad", rel_fro=GRAD_REL_FRO, rel_max=GRAD_REL_MAX):
     err = float(np.max(np.abs(g - ref))) if ref.size else 0.0
     nref = float(np.linalg.norm(ref))
     fro = float(np.linalg.norm(g - ref)) / nref if nref > 0 else float(np.linalg.norm(g))
+    report = os.environ.get("NSA_GRAD_REPORT")
+    if report:
+        with open(report, "a") as f:
+            f.write(json.dumps({"name": name, "rel_max": err / scale if scale > 0 else 0.0, "rel_fro": fro,
+                                "test": os.environ.get("PYTEST_CURRENT_TEST", "")}) + "\n")
     assert err <= rel_max * scale + 1e-6, f"{name}: max-abs error {err} > {rel_max} x {scale}"
     assert fro <= rel_fro or nref == 0 and fro <= 1e-6, f"{name}: relative Frobenius error {fro} > {rel_fro}"
     return {"maxabs": err, "scale": scale, "rel_fro": fro}

@@ -49,10 +49,14 @@ def _layout(B, Hq, Hkv, Sq, Skv, D, bq=128, bkv=64, hs=False):
     # when the pooled keys of a head exceed 64 KB and the row has at most
     # 2048 tiles
     nkp = -(-NK // 128) * 128
-    tc = a(B * Hs * NQ * nkp * 4) if (NK * D * 4 > 64 * 1024 and nkp <= 2048) else 0
+    use_tc = NK * D * 4 > 64 * 1024 and nkp <= 2048
+    tc = a(B * Hs * NQ * nkp * 4) if use_tc else 0
+    # and the tf32 hi and lo parts of the scored keys (Hkv heads, or the
+    # one head mean)
+    split = 2 * a(B * (1 if hs else Hkv) * NK * D * 4) if use_tc else 0
     fwd = 256 + a(B * Hkv * 4) + a(B * Hq * NQ * D * 4) + a(B * Hkv * NK * D * 4) + means \
-        + a(B * Hs * NQ * 4) + a(B * Hs * NQ * NK * 2) + tc
-    sel = 256 + means + tc
+        + a(B * Hs * NQ * 4) + a(B * Hs * NQ * NK * 2) + tc + split
+    sel = 256 + means + tc + split
     NQa, NKa = -(-Sq // 128), -(-Skv // 64)
     att = 256 + a(B * Hq * NQa * 4) + a(B * Hq * NQa * NKa * 2)
     return max(fwd, sel, att)

@@ -100,7 +100,7 @@ _lib.nsa_block_sparse_attn_bwd_masked.restype = _I
 _lib.nsa_block_sparse_attn_bwd_masked.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _I, _I, _I,
                                                   _P, _PI64, _F, _P, _P, _P, _P, _SZ, _P]
 _lib.nsa_score_tc.restype = _I
-_lib.nsa_score_tc.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P]
+_lib.nsa_score_tc.argtypes = [_P, _P, _I, _I, _I, _I, _I, _I, _P, _P, _SZ, _P]
 _lib.nsa_bwd_workspace_bytes.restype = _SZ
 _lib.nsa_bwd_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I, _I]
 _lib.nsa_forward.restype = _I
@@ -274,7 +274,10 @@ def nsa_score_tc(pq: torch.Tensor, pk: torch.Tensor, stream=None) -> torch.Tenso
     Hkv, NK = pk.shape[1], pk.shape[2]
     nkp = (NK + 127) // 128 * 128
     out = torch.zeros(B, Hq, NQ, nkp, dtype=torch.float32, device=pq.device)
-    _check(_lib.nsa_score_tc(_ptr(pq), _ptr(pk), B, Hq, Hkv, NQ, NK, D, _ptr(out), _stream(stream)))
+    half = (B * Hkv * NK * D * 4 + 255) // 256 * 256
+    ws = torch.empty(2 * half, dtype=torch.uint8, device=pq.device)
+    _check(_lib.nsa_score_tc(_ptr(pq), _ptr(pk), B, Hq, Hkv, NQ, NK, D, _ptr(out), _ptr(ws), ws.numel(),
+                             _stream(stream)))
     return out[..., :NK]
 
 

@@ -107,6 +107,23 @@ nsa_status encode_tokens(CUtensorMap *map, const void *ptr, int D, int S, long l
   return NSA_OK;
 }
 
+// float32 (BH, N, D) viewed as 3-D {D, N, BH}; box {32, rows, 1} (128-byte
+// rows), 128-byte swizzle. Rows past N read as zero.
+nsa_status encode_f32_rows(CUtensorMap *map, const void *ptr, int D, int N, long long BH, int rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  nsa_status st = get_encoder(&enc);
+  if (st != NSA_OK) return st;
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)N * D * 4};
+  cuuint32_t box[3] = {32, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NSA_ERR_CUDA, "cuTensorMapEncodeTiled (float32) failed (%d)", (int)r);
+  return NSA_OK;
+}
+
 inline long long cdiv(long long a, long long b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 inline bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -150,9 +167,16 @@ size_t tc_scores_bytes(int B, int Hs, int NQ, int NK, int D) {
   const size_t nkp = (size_t)((NK + 127) / 128 * 128);
   return (size_t)B * Hs * NQ * nkp * 4;
 }
+// The tf32 hi and lo parts of the scored keys (Hk kv heads: Hkv, or 1 for
+// head-shared scoring), two float32 arrays shaped like them.
+size_t tc_split_half(int B, int Hk, int NK, int D) { return (size_t)B * Hk * NK * D * 4; }
+size_t tc_split_bytes(int B, int Hk, int NK, int D) {
+  if (!nsa::select_uses_tc_scores(NK, D, 0)) return 0;
+  return 2 * align256(tc_split_half(B, Hk, NK, D));
+}
 
 struct ForwardLayout {
-  size_t flags, counters, pq, pk, qm, km, count, index, tc, total;
+  size_t flags, counters, pq, pk, qm, km, count, index, tc, tcsplit, total;
 };
 ForwardLayout forward_layout(const Geometry &g, bool head_shared) {
   ForwardLayout L;
@@ -175,20 +199,23 @@ ForwardLayout forward_layout(const Geometry &g, bool head_shared) {
   off += align256((size_t)g.B * g.Hs * g.NQ * g.NK * 2);
   L.tc = off;
   off += align256(tc_scores_bytes(g.B, g.Hs, g.NQ, g.NK, g.D));
+  L.tcsplit = off;
+  off += tc_split_bytes(g.B, head_shared ? 1 : g.Hkv, g.NK, g.D);
   L.total = off;
   return L;
 }
 // nsa_select: flag word, then the head means when head_shared
 struct SelectLayout {
-  size_t flags, qm, km, tc, total;
+  size_t flags, qm, km, tc, tcsplit, total;
 };
-SelectLayout select_layout(int B, int Hq, int NQ, int NK, int D, bool head_shared) {
+SelectLayout select_layout(int B, int Hq, int Hkv, int NQ, int NK, int D, bool head_shared) {
   SelectLayout L;
   L.flags = 0;
   L.qm = 256;
   L.km = L.qm + (head_shared ? align256((size_t)B * NQ * D * 4) : 0);
   L.tc = L.km + (head_shared ? align256((size_t)B * NK * D * 4) : 0);
-  L.total = L.tc + align256(tc_scores_bytes(B, head_shared ? 1 : Hq, NQ, NK, D));
+  L.tcsplit = L.tc + align256(tc_scores_bytes(B, head_shared ? 1 : Hq, NQ, NK, D));
+  L.total = L.tcsplit + tc_split_bytes(B, head_shared ? 1 : Hkv, NK, D);
   return L;
 }
 struct AttnLayout {
@@ -281,6 +308,23 @@ nsa_status run_attention(const void *q, const void *k, const void *v, const Geom
   return NSA_OK;
 }
 
+// Long rows: the tf32 split of the pooled keys into `split` (tc_split_bytes),
+// then the scores (B, Hq, NQ, NKP) of pq (B, Hq, NQ, D) against pk (B, Hkv,
+// NK, D) on the tensor cores into `scores`.
+nsa_status run_tc_scores(const float *pq, const float *pk, int B, int Hq, int Hkv, int NQ, int NK, int D,
+                         float *scores, char *split, DeviceInfo *dev, cudaStream_t s) {
+  float *hi = reinterpret_cast<float *>(split);
+  float *lo = reinterpret_cast<float *>(split + align256(tc_split_half(B, Hkv, NK, D)));
+  NSA_CUDA(nsa::launch_split_tf32(pk, (long long)B * Hkv * NK * D, hi, lo, dev->num_sms, s));
+  CUtensorMap thi, tlo;
+  nsa_status st;
+  if ((st = encode_f32_rows(&thi, hi, D, NK, (long long)B * Hkv, 256)) != NSA_OK) return st;
+  if ((st = encode_f32_rows(&tlo, lo, D, NK, (long long)B * Hkv, 256)) != NSA_OK) return st;
+  const nsa::ScoreTcArgs a = {pq, pk, B, Hq, Hkv, NQ, NK, (int)cdiv(NK, 128) * 128, D, 1, scores, dev->err};
+  NSA_CUDA(nsa::launch_score_tc(a, thi, tlo, dev->num_sms, s));
+  return NSA_OK;
+}
+
 nsa::SelectArgs select_args(const float *pq, const float *pk, const Geometry &g, const nsa_spec *spec,
                             const int8_t *pins, const int64_t *ps, const int8_t *drops, const int64_t *ds) {
   nsa::SelectArgs a = {};
@@ -356,18 +400,20 @@ nsa_status nsa_score(const float *pq, const float *pk, int B, int Hq, int Hkv, i
 }
 
 nsa_status nsa_score_tc(const float *pq, const float *pk, int B, int Hq, int Hkv, int NQ, int NK, int D,
-                        float *scores, nsa_stream_t stream) {
+                        float *scores, void *workspace, size_t workspace_bytes, nsa_stream_t stream) {
   g_last_error.clear();
-  if (!pq || !pk || !scores) return fail(NSA_ERR_INVALID_ARG, "nsa_score_tc: NULL pointer");
+  if (!pq || !pk || !scores || !workspace) return fail(NSA_ERR_INVALID_ARG, "nsa_score_tc: NULL pointer");
   nsa_status st = check_dims(B, Hq, Hkv, NQ, NK, D);
   if (st != NSA_OK) return st;
-  if (!aligned(pq, 16) || !aligned(pk, 16) || !aligned(scores, 16))
-    return fail(NSA_ERR_INVALID_ARG, "nsa_score_tc: pq, pk, scores must be 16-byte aligned");
+  if (!aligned(pq, 16) || !aligned(pk, 16) || !aligned(scores, 16) || !aligned(workspace, 256))
+    return fail(NSA_ERR_INVALID_ARG, "nsa_score_tc: pq, pk, scores must be 16-byte aligned, workspace 256");
+  const size_t need = 2 * align256(tc_split_half(B, Hkv, NK, D));
+  if (workspace_bytes < need)
+    return fail(NSA_ERR_INVALID_ARG, "nsa_score_tc: workspace needs %zu bytes (got %zu)", need, workspace_bytes);
   DeviceInfo *dev;
   if ((st = device_info(&dev)) != NSA_OK) return st;
-  const nsa::ScoreTcArgs a = {pq, pk, B, Hq, Hkv, NQ, NK, (int)cdiv(NK, 128) * 128, D, 1, scores, dev->err};
-  NSA_CUDA(nsa::launch_score_tc(a, dev->num_sms, (cudaStream_t)stream));
-  return NSA_OK;
+  return run_tc_scores(pq, pk, B, Hq, Hkv, NQ, NK, D, scores, static_cast<char *>(workspace), dev,
+                       (cudaStream_t)stream);
 }
 
 nsa_status nsa_select(const float *pq, const float *pk, int B, int Hq, int Hkv, int NQ, int NK, int D,
@@ -385,7 +431,7 @@ nsa_status nsa_select(const float *pq, const float *pk, int B, int Hq, int Hkv, 
   if (!aligned(pq, 16) || !aligned(pk, 16) || !aligned(workspace, 256) || !aligned(kv_count, 4) ||
       !aligned(kv_index, 2))
     return fail(NSA_ERR_INVALID_ARG, "nsa_select: misaligned pointer");
-  const SelectLayout L = select_layout(B, Hq, NQ, NK, D, spec->head_shared != 0);
+  const SelectLayout L = select_layout(B, Hq, Hkv, NQ, NK, D, spec->head_shared != 0);
   if (workspace_bytes < L.total)
     return fail(NSA_ERR_INVALID_ARG, "nsa_select: workspace needs %zu bytes (got %zu)", L.total, workspace_bytes);
   Geometry g = {B, Hq, Hkv, 0, 0, D, NQ, NK, spec->head_shared ? 1 : Hq};
@@ -415,7 +461,11 @@ nsa_status nsa_select(const float *pq, const float *pk, int B, int Hq, int Hkv, 
   a.kv_index = kv_index;
   a.not_covered = flag;
   a.err = dev->err;
-  if (tc_scores_bytes(B, g.Hs, NQ, NK, D) > 0) a.tc_scores = reinterpret_cast<float *>(ws + L.tc);
+  if (tc_scores_bytes(B, g.Hs, NQ, NK, D) > 0) {
+    a.tc_scores = reinterpret_cast<float *>(ws + L.tc);
+    if ((st = run_tc_scores(a.pq, a.pk, B, a.Hq, a.Hkv, NQ, NK, D, a.tc_scores, ws + L.tcsplit, dev, s)) != NSA_OK)
+      return st;
+  }
   NSA_CUDA(nsa::launch_select(a, dev->num_sms, s));
   *is_dense = 0;
   if (!spec->force) {
@@ -605,7 +655,11 @@ nsa_status forward_impl(const void *q, const void *k, const void *v, int B, int 
   a.kv_index = index;
   a.not_covered = plan ? nullptr : flag;
   a.err = dev->err;
-  if (tc_scores_bytes(B, g.Hs, NQ, NK, D) > 0) a.tc_scores = reinterpret_cast<float *>(ws + L.tc);
+  if (tc_scores_bytes(B, g.Hs, NQ, NK, D) > 0) {
+    a.tc_scores = reinterpret_cast<float *>(ws + L.tc);
+    if ((st = run_tc_scores(a.pq, a.pk, B, a.Hq, a.Hkv, NQ, NK, D, a.tc_scores, ws + L.tcsplit, dev, s)) != NSA_OK)
+      return st;
+  }
   NSA_CUDA(nsa::launch_select(a, dev->num_sms, s));
   NSA_CUDA(mark(2));
   // 3. attention over kept tiles; without a plan, dense when the device flag
@@ -645,7 +699,7 @@ size_t nsa_workspace_bytes(int B, int Hq, int Hkv, int Sq, int Skv, int D, const
   const bool hs = spec->head_shared != 0;
   Geometry g = {B, Hq, Hkv, Sq, Skv, D, NQ, NK, hs ? 1 : Hq};
   size_t f = forward_layout(g, hs).total;
-  const size_t sel = select_layout(B, Hq, NQ, NK, D, hs).total;
+  const size_t sel = select_layout(B, Hq, Hkv, NQ, NK, D, hs).total;
   const int NQa = (int)cdiv(Sq, 128), NKa = (int)cdiv(Skv, 64);
   const size_t at = attn_layout(B, Hq, NQa, NKa).total;
   if (sel > f) f = sel;

@@ -91,15 +91,18 @@ struct SelectArgs {
   const int32_t *plan_k;
   long long plan_bs, plan_hs;  // tile-row strides (rows of NK) per batch / head
   // when set (rows whose pooled keys do not fit beside the scoring CTA):
-  // the scores are computed on the tensor cores into this scratch, (B, Hs,
-  // NQ, NKP) float32 with NKP = NK rounded up to 128, and the top-k reads
-  // them from there
+  // the scores were computed on the tensor cores (launch_score_tc) into this
+  // scratch, (B, Hs, NQ, NKP) float32 with NKP = NK rounded up to 128, and
+  // the top-k reads them from there
   float *tc_scores;
 };
 
 // Pooled scores on the tensor cores (score_tc.cu): scores (B, Hq, NQ, NKP)
 // = pq (B, Hq, NQ, D) . pk (B, Hkv, NK, D)^T, query head h against kv head
-// h / (Hq / Hkv); columns from NK up to the next multiple of 64 hold zeros.
+// h / (Hq / Hkv); columns from NK up to NKP hold zeros. The keys come as
+// their tf32 hi and lo parts (launch_split_tf32), read through the tensor
+// maps thi / tlo: {D, NK, B*Hkv} float32, boxes {32, 256, 1}, 128-byte
+// swizzle.
 struct ScoreTcArgs {
   const float *pq;
   const float *pk;
@@ -108,8 +111,12 @@ struct ScoreTcArgs {
   float *scores;
   unsigned int *err;
 };
-cudaError_t launch_score_tc(ScoreTcArgs a, int num_sms, cudaStream_t stream);
+cudaError_t launch_score_tc(ScoreTcArgs a, const CUtensorMap &thi, const CUtensorMap &tlo, int num_sms,
+                            cudaStream_t stream);
 size_t score_tc_smem(int D);
+// hi = tf32(x), lo = tf32(x - hi) elementwise (n a multiple of 4, 16-byte
+// aligned arrays).
+cudaError_t launch_split_tf32(const float *x, long long n, float *hi, float *lo, int num_sms, cudaStream_t stream);
 // True when launch_select computes the scores of these rows on the tensor
 // cores (given a scratch): the pooled keys of a head do not fit in the
 // resident path and the row fits the register top-k (NK <= 2048).

@@ -11,13 +11,18 @@
 // peak performance", 2022); the dropped lo.lo term and the roundings leave a
 // relative error near 2^-21 per product, the size of float32 FMA rounding.
 //
-// One CTA: 128 pooled query rows (M) of one keep head against a range of
-// 64-row pooled key chunks (N = 64, K = D). The query halves stay in shared
-// memory; each key chunk is loaded into registers while the previous chunk's
-// products run, split, and stored in 128-byte swizzled K-major tiles. The
-// accumulator is double-buffered in TMEM; warps 4-7 (one query row per
-// thread) copy a finished chunk's 64 scores per row to the score scratch
-// while the next chunk is multiplied. Every wait is bounded.
+// The pooled keys of every kv head are split once (split_tf32_kernel) into
+// two float32 arrays laid out like pk. One CTA then takes 128 pooled query
+// rows (M) of one keep head: its epilogue warps split those rows and store
+// hi and lo in TMEM, where they are the A operand of every MMA, so the
+// whole shared memory holds key tiles. The keys stream in by TMA in chunks
+// of 256 kv tiles (N = 256: one MMA instruction does four times the work of
+// an N = 64 one, and issuing MMAs, not executing them, is what bounds a
+// single issuing thread), one 32-element segment of the head dimension (hi
+// and lo, 64 KB) per ring stage. Per segment 4 K-steps x 3 products go into
+// a 256-column f32 accumulator in TMEM; the epilogue warps (one query row
+// per thread) copy each finished chunk to the score scratch and free the
+// accumulator for the next chunk. Every wait is bounded.
 #include <algorithm>
 
 #include "nsa_device.cuh"
@@ -27,54 +32,27 @@ namespace nsa {
 
 namespace {
 
-constexpr int TM = 128;  // query rows per CTA (the MMA's M)
-constexpr int TN = 64;   // kv tiles per chunk (the MMA's N)
-constexpr int kTcThreads = 256;
-
-template <int D>
-struct TcCfg {
-  static constexpr int Q_BYTES = TM * D * 4;
-  static constexpr int K_BYTES = TN * D * 4;
-  static constexpr int OFF_QH = 0;
-  static constexpr int OFF_QL = Q_BYTES;
-  static constexpr int OFF_KH = 2 * Q_BYTES;
-  static constexpr int OFF_KL = OFF_KH + K_BYTES;
-  static constexpr int OFF_BAR = OFF_KL + K_BYTES;
-  static constexpr int TILE_BYTES = OFF_BAR + 64;
-  static constexpr int SMEM_BYTES = TILE_BYTES + 1024;  // room to align the base to 1024
-  static constexpr int UNITS_PER_ROW = D / 4;           // 16-byte units (4 floats)
-  static constexpr int K_UNITS = TN * UNITS_PER_ROW / kTcThreads;  // per thread
-};
+constexpr int TM = 128;                          // query rows per CTA (the MMA's M)
+constexpr int TN = 256;                          // kv tiles per chunk (the MMA's N)
+constexpr int KSEG = 32;                         // f32 elements of D per 128-byte row
+constexpr int KST = 3;                           // ring stages
+constexpr int SEG_BYTES = TN * 128;              // one D segment of a chunk, hi or lo (32 KB)
+constexpr int STAGE_BYTES = 2 * SEG_BYTES;       // hi, then lo
+constexpr int OFF_BAR = KST * STAGE_BYTES;       // 192 KB of key tiles
+constexpr int TILE_BYTES = OFF_BAR + 256;
+constexpr int kTcThreads = 192;                  // 6 warps
+constexpr uint32_t COL_QHI = 0, COL_QLO = 128, COL_ACC = 256, TMEM_COLS = 512;
 
 struct TcBars {
-  uint64_t acc_full[2];
+  uint64_t full[KST];
+  uint64_t empty[KST];
+  uint64_t q_ready;    // the epilogue warps stored the split query rows (4 arrivals)
+  uint64_t acc_full;   // a chunk's products completed
+  uint64_t acc_empty;  // the epilogue copied the chunk out (4 arrivals)
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
-
-// Byte offset of 16-byte unit k4 (floats 4 k4 .. 4 k4 + 3) of row r in a
-// K-major tile of R rows with 128-byte swizzle: 32 floats per 128-byte row
-// segment, segment s of every row at s * R * 128, rows 128 bytes apart, the
-// unit's position within the row XORed with (r & 7).
-__device__ __forceinline__ uint32_t sw_off(int R, int r, int k4) {
-  return (uint32_t)((k4 >> 3) * R * 128 + r * 128 + (((k4 & 7) ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ void split_store(unsigned char *hi_tile, unsigned char *lo_tile, uint32_t off,
-                                            const float4 &v) {
-  uint4 h, l;
-  h.x = to_tf32(v.x);
-  h.y = to_tf32(v.y);
-  h.z = to_tf32(v.z);
-  h.w = to_tf32(v.w);
-  l.x = to_tf32(v.x - __uint_as_float(h.x));
-  l.y = to_tf32(v.y - __uint_as_float(h.y));
-  l.z = to_tf32(v.z - __uint_as_float(h.z));
-  l.w = to_tf32(v.w - __uint_as_float(h.w));
-  *reinterpret_cast<uint4 *>(hi_tile + off) = h;
-  *reinterpret_cast<uint4 *>(lo_tile + off) = l;
-}
 
 __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned int *err,
                                           unsigned int site) {
@@ -85,25 +63,42 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
   return ok != 0;
 }
 
+__global__ void split_tf32_kernel(const float4 *x, long long n4, float4 *hi, float4 *lo) {
+  pdl_wait();  // the pooled keys come from the previous kernel
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    const float4 v = x[i];
+    float4 h, l;
+    h.x = __uint_as_float(to_tf32(v.x));
+    h.y = __uint_as_float(to_tf32(v.y));
+    h.z = __uint_as_float(to_tf32(v.z));
+    h.w = __uint_as_float(to_tf32(v.w));
+    l.x = __uint_as_float(to_tf32(v.x - h.x));
+    l.y = __uint_as_float(to_tf32(v.y - h.y));
+    l.z = __uint_as_float(to_tf32(v.z - h.z));
+    l.w = __uint_as_float(to_tf32(v.w - h.w));
+    hi[i] = h;
+    lo[i] = l;
+  }
+}
+
 template <int D>
-__global__ void __launch_bounds__(kTcThreads, 1) score_tc_kernel(const ScoreTcArgs a) {
-  using C = TcCfg<D>;
-  constexpr int UPR = C::UNITS_PER_ROW;
+__global__ void __launch_bounds__(kTcThreads, 1)
+    score_tc_kernel(const ScoreTcArgs a, const __grid_constant__ CUtensorMap thi,
+                    const __grid_constant__ CUtensorMap tlo) {
+  constexpr int NSEG = D / KSEG;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_u32 & 1023u)) & 1023u;
   uint32_t dyn_size;
   asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_size));
-  if (pad + C::TILE_BYTES > dyn_size) {
+  if (pad + TILE_BYTES > dyn_size) {
     if (threadIdx.x == 0) atomicOr(a.err, kErrSmemLayout);
     return;
   }
   unsigned char *smem = smem_raw + pad;
-  unsigned char *sQH = smem + C::OFF_QH, *sQL = smem + C::OFF_QL;
-  unsigned char *sKH = smem + C::OFF_KH, *sKL = smem + C::OFF_KL;
-  TcBars *bars = reinterpret_cast<TcBars *>(smem + C::OFF_BAR);
+  TcBars *bars = reinterpret_cast<TcBars *>(smem + OFF_BAR);
   volatile int *abort = &bars->abort;
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
 
   const int rb = blockIdx.x, hs = blockIdx.y;
   const int b = blockIdx.z / a.nsplit, sp = blockIdx.z % a.nsplit;
@@ -112,147 +107,182 @@ __global__ void __launch_bounds__(kTcThreads, 1) score_tc_kernel(const ScoreTcAr
   const int per = (nchunks + a.nsplit - 1) / a.nsplit;
   const int c0 = sp * per, c1 = min(nchunks, c0 + per);
 
-  if (tid == 0) {
-    mbar_init(&bars->acc_full[0], 1);
-    mbar_init(&bars->acc_full[1], 1);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < KST; ++s) {
+      mbar_init(&bars->full[s], 1);
+      mbar_init(&bars->empty[s], 1);
+    }
+    mbar_init(&bars->q_ready, 4);
+    mbar_init(&bars->acc_full, 1);
+    mbar_init(&bars->acc_empty, 4);
     mbar_init(&bars->drain, 1);
     bars->abort = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(&bars->tmem_base, 2 * TN);
+  if (warp == 1) tmem_alloc(&bars->tmem_base, TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  pdl_wait();  // the pooled vectors come from the previous kernels
+  pdl_wait();  // the pooled vectors and their split come from the previous kernels
 
-  // ---- the CTA's 128 query rows, split into tf32 halves (rows past NQ: 0)
-  const int nrows = min(TM, a.NQ - rb * TM);
-  const float *qb = a.pq + (((size_t)b * a.Hq + hs) * a.NQ + (size_t)rb * TM) * D;
-  for (int u = tid; u < TM * UPR; u += kTcThreads) {
-    const int r = u / UPR, k4 = u % UPR;
-    const float4 v = r < nrows ? *reinterpret_cast<const float4 *>(qb + (size_t)r * D + k4 * 4)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-    split_store(sQH, sQL, sw_off(TM, r, k4), v);
-  }
-
-  // ---- key chunks: loaded into registers one chunk ahead
-  const float *kb = a.pk + ((size_t)b * a.Hkv + hk) * (size_t)a.NK * D;
-  float4 kreg[C::K_UNITS];
-  auto load_chunk = [&](int c) {
-#pragma unroll
-    for (int it = 0; it < C::K_UNITS; ++it) {
-      const int u = tid + it * kTcThreads;
-      const int r = u / UPR, k4 = u % UPR;
-      const int j = c * TN + r;
-      kreg[it] = j < a.NK ? *reinterpret_cast<const float4 *>(kb + (size_t)j * D + k4 * 4)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+  if (warp == 0) {
+    // ----------------------------------------------------------- producer
+    if (lane == 0 && c0 < c1) {
+      tma_prefetch_desc(&thi);
+      tma_prefetch_desc(&tlo);
+      int it = 0;
+      for (int c = c0; c < c1 && !*abort; ++c) {
+        for (int sg = 0; sg < NSEG; ++sg, ++it) {
+          const int st = it % KST;
+          if (it >= KST && !mbar_wait(&bars->empty[st], ((it / KST) - 1) & 1, abort, a.err, 0x60)) break;
+          mbar_arrive_expect_tx(&bars->full[st], STAGE_BYTES);
+          unsigned char *dst = smem + st * STAGE_BYTES;
+          tma_load_3d(dst, &thi, &bars->full[st], sg * KSEG, c * TN, b * a.Hkv + hk);
+          tma_load_3d(dst + SEG_BYTES, &tlo, &bars->full[st], sg * KSEG, c * TN, b * a.Hkv + hk);
+        }
+      }
+      if (*abort) {
+        // wait (bounded, ignoring the abort flag) for copies still in flight
+        int never = 0;
+        for (int m = (it > KST ? it - KST : 0); m < it; ++m)
+          mbar_wait(&bars->full[m % KST], (m / KST) & 1, &never, a.err, 0x61);
+      }
     }
-  };
-  auto store_chunk = [&]() {
+    __syncwarp();
+  } else if (warp == 1) {
+    // --------------------------------------------------------- MMA issuer
+    if (lane == 0 && c0 < c1) {
+      constexpr uint32_t idesc = idesc_tf32_f32(TM, TN);
+      const uint64_t dk = smem_desc_sw128(smem_u32(smem), 16, 1024);
+      bool ok = mbar_wait(&bars->q_ready, 0, abort, a.err, 0x62);
+      int it = 0;
+      for (int c = c0; ok && c < c1; ++c) {
+        if (c > c0 && !mbar_wait(&bars->acc_empty, (c - c0 - 1) & 1, abort, a.err, 0x63)) {
+          ok = false;
+          break;
+        }
+        for (int sg = 0; sg < NSEG; ++sg, ++it) {
+          const int st = it % KST;
+          if (!mbar_wait(&bars->full[st], (it / KST) & 1, abort, a.err, 0x64)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t dhi = dk + ((uint64_t)(st * STAGE_BYTES) >> 4);
+          const uint64_t dlo = dhi + ((uint64_t)SEG_BYTES >> 4);
 #pragma unroll
-    for (int it = 0; it < C::K_UNITS; ++it) {
-      const int u = tid + it * kTcThreads;
-      split_store(sKH, sKL, sw_off(TN, u / UPR, u % UPR), kreg[it]);
+          for (int kk = 0; kk < KSEG / 8; ++kk) {
+            const uint32_t qc = (uint32_t)(sg * KSEG + kk * 8);
+            const uint64_t ko = (uint64_t)((kk * 32) >> 4);
+            umma_tf32_ts(tmem + COL_ACC, tmem + COL_QHI + qc, dhi + ko, idesc, (sg > 0 || kk > 0) ? 1u : 0u);
+            umma_tf32_ts(tmem + COL_ACC, tmem + COL_QHI + qc, dlo + ko, idesc, 1u);
+            umma_tf32_ts(tmem + COL_ACC, tmem + COL_QLO + qc, dhi + ko, idesc, 1u);
+          }
+          umma_commit(&bars->empty[st]);
+        }
+        if (!ok) break;
+        umma_commit(&bars->acc_full);
+      }
+      // every product has completed before TMEM is released
+      umma_commit(&bars->drain);
+      int never = 0;
+      mbar_wait(&bars->drain, 0, &never, a.err, 0x65);
     }
-  };
-  // warps 4-7: the 64 scores of chunk c of each query row, from TMEM buffer bb
-  auto epilogue = [&](int c, int bb) {
+    __syncwarp();
+  } else {
+    // ------------------------------------- query split and score epilogue
+    // (warps 2-5: TMEM lane quarter warp & 3, one query row per thread)
     const int quarter = warp & 3, row = quarter * 32 + lane;
-    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(bb * TN);
-    uint32_t r0[32], r1[32];
-    tmem_ld32(taddr, r0);
-    tmem_ld32(taddr + 32, r1);
-    tmem_wait_ld();
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const int i = rb * TM + row;
-    if (i < a.NQ) {
-      float *dst = a.scores + (((size_t)b * a.Hq + hs) * a.NQ + i) * a.NKP + (size_t)c * TN;
-      uint4 *d4 = reinterpret_cast<uint4 *>(dst);
+    const float *qrow = a.pq + (((size_t)b * a.Hq + hs) * a.NQ + (i < a.NQ ? i : 0)) * D;
 #pragma unroll
-      for (int q = 0; q < 8; ++q) d4[q] = make_uint4(r0[4 * q], r0[4 * q + 1], r0[4 * q + 2], r0[4 * q + 3]);
+    for (int s0 = 0; s0 < D; s0 += 32) {
+      uint32_t h[32], l[32];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) d4[8 + q] = make_uint4(r1[4 * q], r1[4 * q + 1], r1[4 * q + 2], r1[4 * q + 3]);
+      for (int u = 0; u < 8; ++u) {
+        const float4 v = i < a.NQ ? *reinterpret_cast<const float4 *>(qrow + s0 + 4 * u)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          h[4 * u + e] = to_tf32(vv[e]);
+          l[4 * u + e] = to_tf32(vv[e] - __uint_as_float(h[4 * u + e]));
+        }
+      }
+      tmem_st32(lane_base + COL_QHI + s0, h);
+      tmem_st32(lane_base + COL_QLO + s0, l);
     }
-  };
-
-  constexpr uint32_t idesc = idesc_tf32_f32(TM, TN);
-  const uint64_t dQH = smem_desc_sw128(smem_u32(sQH), 16, 1024), dQL = smem_desc_sw128(smem_u32(sQL), 16, 1024);
-  const uint64_t dKH = smem_desc_sw128(smem_u32(sKH), 16, 1024), dKL = smem_desc_sw128(smem_u32(sKL), 16, 1024);
-  bool ok = true;
-  if (c0 < c1) load_chunk(c0);
-  for (int c = c0; c < c1; ++c) {
-    const int n = c - c0, bf = n & 1;
-    // the previous chunk's products have completed (waited below): the key
-    // tiles and accumulator buffer bf are free
-    store_chunk();
-    fence_proxy_async_smem();
+    tmem_wait_st();
     tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    if (tid == 0) {
-      const uint32_t d_tmem = tmem + (uint32_t)(bf * TN);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars->q_ready);
+    for (int c = c0; c < c1; ++c) {
+      if (!warp_wait(&bars->acc_full, (c - c0) & 1, abort, a.err, 0x66)) break;
+      tc_fence_after();
+      float *dst = a.scores + (((size_t)b * a.Hq + hs) * a.NQ + i) * a.NKP;
+#pragma unroll 2
+      for (int part = 0; part < TN / 32; ++part) {
+        uint32_t r[32];
+        tmem_ld32(lane_base + COL_ACC + part * 32, r);
+        tmem_wait_ld();
+        const int col = c * TN + part * 32;
+        if (i < a.NQ && col < a.NKP) {
+          uint4 *d4 = reinterpret_cast<uint4 *>(dst + col);
 #pragma unroll
-      for (int kk = 0; kk < D / 8; ++kk) {
-        const uint32_t oq = (kk / 4) * (TM * 128) + (kk % 4) * 32, ok_ = (kk / 4) * (TN * 128) + (kk % 4) * 32;
-        umma_tf32_ss(d_tmem, dQH + (oq >> 4), dKH + (ok_ >> 4), idesc, kk > 0 ? 1u : 0u);
+          for (int q = 0; q < 8; ++q) d4[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+        }
       }
-#pragma unroll
-      for (int kk = 0; kk < D / 8; ++kk) {
-        const uint32_t oq = (kk / 4) * (TM * 128) + (kk % 4) * 32, ok_ = (kk / 4) * (TN * 128) + (kk % 4) * 32;
-        umma_tf32_ss(d_tmem, dQH + (oq >> 4), dKL + (ok_ >> 4), idesc, 1u);
-      }
-#pragma unroll
-      for (int kk = 0; kk < D / 8; ++kk) {
-        const uint32_t oq = (kk / 4) * (TM * 128) + (kk % 4) * 32, ok_ = (kk / 4) * (TN * 128) + (kk % 4) * 32;
-        umma_tf32_ss(d_tmem, dQL + (oq >> 4), dKH + (ok_ >> 4), idesc, 1u);
-      }
-      umma_commit(&bars->acc_full[bf]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->acc_empty);
     }
-    if (c + 1 < c1) load_chunk(c + 1);
-    if (n >= 1 && warp >= 4) epilogue(c - 1, bf ^ 1);
-    if (!warp_wait(&bars->acc_full[bf], (n >> 1) & 1, abort, a.err, 0x60)) {
-      ok = false;
-      break;
-    }
-    tc_fence_after();
-  }
-  if (ok && c1 > c0 && warp >= 4) epilogue(c1 - 1, (c1 - c0 - 1) & 1);
-  if (tid == 0) {
-    // every product has completed before TMEM is released
-    umma_commit(&bars->drain);
-    int never = 0;
-    mbar_wait(&bars->drain, 0, &never, a.err, 0x61);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 2 * TN);
+  if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
 }
 
 }  // namespace
 
-size_t score_tc_smem(int D) { return D == 64 ? TcCfg<64>::SMEM_BYTES : TcCfg<128>::SMEM_BYTES; }
+size_t score_tc_smem(int D) {
+  (void)D;
+  return (size_t)TILE_BYTES;
+}
 
-cudaError_t launch_score_tc(ScoreTcArgs a, int num_sms, cudaStream_t stream) {
+cudaError_t launch_split_tf32(const float *x, long long n, float *hi, float *lo, int num_sms, cudaStream_t stream) {
+  const long long n4 = n / 4;
+  if (n4 == 0) return cudaSuccess;
+  long long blocks = (n4 + 255) / 256;
+  if (blocks > (long long)num_sms * 8) blocks = (long long)num_sms * 8;
+  return launch_pdl(split_tf32_kernel, dim3((unsigned)blocks), dim3(256), 0, stream,
+                    reinterpret_cast<const float4 *>(x), n4, reinterpret_cast<float4 *>(hi),
+                    reinterpret_cast<float4 *>(lo));
+}
+
+cudaError_t launch_score_tc(ScoreTcArgs a, const CUtensorMap &thi, const CUtensorMap &tlo, int num_sms,
+                            cudaStream_t stream) {
   const int nchunks = (a.NK + TN - 1) / TN;
   const long long blocks = (long long)((a.NQ + TM - 1) / TM) * a.Hq * a.B;
   if (blocks == 0 || nchunks == 0) return cudaSuccess;
   // few row blocks: split the kv range so the grid covers the device
   a.nsplit = (int)std::min<long long>(nchunks, std::max<long long>(1, (num_sms + blocks - 1) / blocks));
   const dim3 grid((unsigned)((a.NQ + TM - 1) / TM), (unsigned)a.Hq, (unsigned)(a.B * a.nsplit));
-  const int smem = (int)score_tc_smem(a.D);
+  const int smem = TILE_BYTES;
   cudaError_t e;
   if (a.D == 64) {
     if ((e = cudaFuncSetAttribute(score_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
         cudaSuccess)
       return e;
-    return launch_pdl(score_tc_kernel<64>, grid, dim3(kTcThreads), (size_t)smem, stream, a);
+    return launch_pdl(score_tc_kernel<64>, grid, dim3(kTcThreads), (size_t)smem, stream, a, thi, tlo);
   }
   if ((e = cudaFuncSetAttribute(score_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
       cudaSuccess)
     return e;
-  return launch_pdl(score_tc_kernel<128>, grid, dim3(kTcThreads), (size_t)smem, stream, a);
+  return launch_pdl(score_tc_kernel<128>, grid, dim3(kTcThreads), (size_t)smem, stream, a, thi, tlo);
 }
 
 }  // namespace nsa

@@ -35,6 +35,8 @@
 //     their keys in registers; longer rows keep them in shared memory.
 //  4. keep = (must & ~forbidden) | selected, written as int8, plus the
 //     ascending compacted index list and its count.
+#include <algorithm>
+
 #include "nsa_device.cuh"
 #include "nsa_kernels.cuh"
 
@@ -184,22 +186,10 @@ __device__ __forceinline__ uint32_t warp_kth_largest(uint32_t (&x)[N], int k) {
 // nearly every key into one bin (and its counter). Every lane returns the
 // same value.
 template <int G>
-__device__ __forceinline__ uint32_t warp_kth_radix(const uint32_t (&kk)[G][4], int k) {
+__device__ __forceinline__ uint32_t warp_kth_interval(const uint32_t (&kk)[G][4], int kr, uint32_t lo, uint32_t hi) {
   __shared__ int hist_all[kThreads / 32][256];
   int *hist = hist_all[threadIdx.x / 32];
   const int lane = threadIdx.x & 31;
-  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int e = 0; e < 4; ++e)
-      if (kk[g][e] != 0u) {
-        lo = min(lo, kk[g][e]);
-        hi = max(hi, kk[g][e]);
-      }
-  lo = __reduce_min_sync(0xffffffffu, lo);
-  hi = __reduce_max_sync(0xffffffffu, hi);
-  int kr = k;
 #pragma unroll 1
   while (lo < hi) {
     // bin width 2^shift with (hi - lo) >> shift < 256
@@ -253,6 +243,25 @@ __device__ __forceinline__ uint32_t warp_kth_radix(const uint32_t (&kk)[G][4], i
   return lo;
 }
 
+// The kr-th largest key in [lo, hi] is the answer; the first interval is the
+// keys' own range.
+template <int G>
+__device__ __forceinline__ uint32_t warp_kth_radix(const uint32_t (&kk)[G][4], int k) {
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (kk[g][e] != 0u) {
+        lo = min(lo, kk[g][e]);
+        hi = max(hi, kk[g][e]);
+      }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  return warp_kth_interval<G>(kk, k, lo, hi);
+}
+
+
 // The row's budget count: the plan's, else ceil(f32(c) * f32(budget)).
 __device__ __forceinline__ int row_budget(const SelectArgs &a, int b, int hs, int i, int c) {
   if (a.plan_k) return a.plan_k[b * a.plan_bs + hs * a.plan_hs + i];
@@ -281,12 +290,17 @@ __device__ __forceinline__ void select_rows_regs(const SelectArgs &a, const floa
     uint32_t kk[G][4];
     uint64_t forced = 0;  // bit 4g+e: must and not forbidden
     int c_lane = 0;
+    // every load of the row first, so that they are in flight together
+    float4 svs[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+      // groups past the row stride NKP (a multiple of 128) hold no tiles
+      svs[g] = g * 128 < NKP ? *reinterpret_cast<const float4 *>(ss + (size_t)r * NKP + g * 128 + lane * 4)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const int jb = g * 128 + lane * 4;
-      // groups past the row stride NKP (a multiple of 128) hold no tiles
-      const float4 sv = g * 128 < NKP ? *reinterpret_cast<const float4 *>(ss + (size_t)r * NKP + jb)
-                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float4 sv = svs[g];
       const float sa[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -304,7 +318,9 @@ __device__ __forceinline__ void select_rows_regs(const SelectArgs &a, const floa
     }
     const int c = __reduce_add_sync(0xffffffffu, c_lane);
     const int k = row_budget(a, b, hs, i, c);
-    if (lane == 0 && k < c && a.not_covered) atomicOr(a.not_covered, 1u);
+    // (the flag is read first: once set, no row needs to touch it again)
+    if (lane == 0 && k < c && a.not_covered && *reinterpret_cast<volatile unsigned int *>(a.not_covered) == 0u)
+      atomicOr(a.not_covered, 1u);
 
     uint32_t T;
     int take;
@@ -325,7 +341,7 @@ __device__ __forceinline__ void select_rows_regs(const SelectArgs &a, const floa
           for (int e = 0; e < 4; ++e) y[4 * g + e] = kk[g][e];
         T = warp_kth_largest<4 * G>(y, k);
       } else {
-        // long rows: radix selection over 8-bit digits
+        // long rows: repeated bucketing of the key range
         T = warp_kth_radix<G>(kk, k);
       }
       int above = 0;
@@ -420,7 +436,9 @@ __device__ __forceinline__ void select_rows_smem(const SelectArgs &a, float *ss,
     }
     const int c = __reduce_add_sync(0xffffffffu, c_lane);
     const int k = row_budget(a, b, hs, i, c);
-    if (lane == 0 && k < c && a.not_covered) atomicOr(a.not_covered, 1u);
+    // (the flag is read first: once set, no row needs to touch it again)
+    if (lane == 0 && k < c && a.not_covered && *reinterpret_cast<volatile unsigned int *>(a.not_covered) == 0u)
+      atomicOr(a.not_covered, 1u);
     __syncwarp();
 
     uint32_t T;
@@ -825,14 +843,263 @@ __global__ void __launch_bounds__(kThreads) select_fusedq_kernel(SelectArgs a) {
 
 // ------------------------------------------------- from tensor-core scores
 // Plan + top-k + outputs for rows whose scores score_tc_kernel wrote to the
-// scratch (row stride NKP): one warp per row, 8 rows per CTA.
+// scratch (row stride NKP <= 2048): one warp per keep row, four rows per
+// CTA at a time, the row's candidate keys in the warp's slice of shared
+// memory (tile order; few registers, so many warps per SM hide the long
+// dependent chains of a row). Lane l handles the tiles j = l + 32 m: each
+// load and shared-memory access of the warp covers 32 consecutive tiles,
+// and one lane's tiles lie 32 apart.
+// The k-th largest candidate key T: the k-th largest of the warp's group
+// maxima (each lane's tiles in four groups) is a key L with at least k keys
+// >= L (distinct tiles), so T is the k-th largest of the keys >= L. Those,
+// usually a little more than k, are gathered and sorted across the warp
+// (bitonic); when more than 256 keys are >= L (or k > 128), the keys are
+// bucketed by range instead (warp_kth_radix). Ties at T go to the lowest
+// tile indices. Lane l writes the outputs of tiles 64 l .. 64 l + 63.
+constexpr int kSelWarps = 4;
+constexpr int kSelBuf = 256;
+
+// warp_kth_radix for keys held in shared memory (n keys, nonzero = a
+// candidate; lane l reads entries l, l + 32, ...): the same bucketing of
+// the key range, with the counts in the warp's 256-entry scratch `hist`.
+__device__ __noinline__ uint32_t warp_kth_range_smem(const uint32_t *key, int n, int k, uint32_t *hist) {
+  const int lane = threadIdx.x & 31;
+  uint32_t lo = 0xFFFFFFFFu, hi = 0u;
+  for (int q = lane; q < n; q += 32)
+    if (key[q] != 0u) {
+      lo = min(lo, key[q]);
+      hi = max(hi, key[q]);
+    }
+  lo = __reduce_min_sync(0xffffffffu, lo);
+  hi = __reduce_max_sync(0xffffffffu, hi);
+  int kr = k;
+  while (lo < hi) {
+    const int shift = max(0, 24 - __clz(hi - lo));
+    for (int q = lane; q < 256; q += 32) hist[q] = 0u;
+    __syncwarp();
+    for (int q = lane; q < n; q += 32) {
+      const uint32_t kv = key[q];
+      if (kv != 0u && kv >= lo && kv <= hi) atomicAdd(&hist[(kv - lo) >> shift], 1u);
+    }
+    __syncwarp();
+    int c8[8], sum = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      c8[q] = (int)hist[255 - (lane * 8 + q)];
+      sum += c8[q];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    const int excl = incl - sum;
+    const bool mine = excl < kr && kr <= incl;
+    int bin = 0, above = excl;
+    if (mine) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (above + c8[q] >= kr) {
+          bin = 255 - (lane * 8 + q);
+          break;
+        }
+        above += c8[q];
+      }
+    }
+    const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
+    bin = __shfl_sync(0xffffffffu, bin, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    kr -= above;
+    const uint32_t nlo = lo + ((uint32_t)bin << shift);
+    const uint32_t width = (1u << shift) - 1u;
+    hi = (hi - nlo < width) ? hi : nlo + width;
+    lo = nlo;
+    __syncwarp();
+  }
+  return lo;
+}
+
 template <int KPL>
-__global__ void __launch_bounds__(kThreads) select_scores_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(kSelWarps * 32, 6) select_scores_kernel(SelectArgs a) {
+  __shared__ uint32_t skey[kSelWarps][32 * KPL];
+  __shared__ uint32_t sbuf[kSelWarps][kSelBuf];
   pdl_wait();  // the scores come from the previous kernel
-  const int NKP = round_up(a.NK, 128);
-  const int i0 = blockIdx.x * 8, hs = blockIdx.y, b = blockIdx.z;
-  const float *ss = a.tc_scores + (((size_t)b * a.Hs + hs) * a.NQ + i0) * NKP;
-  select_rows_regs<8, KPL>(a, ss, NKP, i0, hs, b);
+  const int NK = a.NK, NQ = a.NQ;
+  const int NKP = round_up(NK, 128);
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  uint32_t *key = skey[warp];
+  uint32_t *buf = sbuf[warp];
+  const long long rows = (long long)a.B * a.Hs * NQ;
+  constexpr int GPL = 4;                      // group maxima per lane (128 per warp)
+  constexpr int MPG = KPL / GPL > 0 ? KPL / GPL : 1;  // tiles per group
+  // keep rows written 16 bytes at a time: the tensor is 16-byte aligned and
+  // rows, NK bytes apart, stay aligned
+  const bool keep16 = a.keep && (NK & 15) == 0 && (reinterpret_cast<uintptr_t>(a.keep) & 15u) == 0;
+  for (long long row = (long long)blockIdx.x * kSelWarps + warp; row < rows; row += (long long)gridDim.x * kSelWarps) {
+    const int i = (int)(row % NQ);
+    const int hs = (int)((row / NQ) % a.Hs);
+    const int b = (int)(row / ((long long)NQ * a.Hs));
+    const RowPlan pl(a, b, hs, i);
+    // rows with no pins, drops or plan: the forced tiles are the diagonal
+    // run [d0, d1] (int compares only)
+    const bool diag_only = !pl.prow && !pl.drow && !pl.srow;
+    const int d0 = (int)pl.jd0, d1 = (int)pl.jd1;
+    auto is_cand = [&](int j) {
+      return diag_only ? (j < d0 || j > d1) : (!pl.must(j) && !pl.forbidden(j));
+    };
+    auto is_forced = [&](int j) { return diag_only ? (j >= d0 && j <= d1) : (pl.must(j) && !pl.forbidden(j)); };
+    const float *ss = a.tc_scores + row * NKP;
+    // keys: 0 for tiles that are not candidates (and past NK)
+    uint32_t gm[GPL] = {0u, 0u, 0u, 0u};
+    int c_lane = 0;
+#pragma unroll
+    for (int g = 0; g < GPL; ++g) {
+      float v[MPG];
+#pragma unroll
+      for (int u = 0; u < MPG; ++u) {
+        const int j = lane + 32 * (g * MPG + u);
+        v[u] = (g * MPG + u < KPL && j < NKP) ? ss[j] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < MPG; ++u) {
+        const int m = g * MPG + u;
+        if (m >= KPL) break;
+        const int j = lane + 32 * m;
+        uint32_t kv = 0u;
+        if (j < NK && is_cand(j)) {
+          kv = order_key(v[u]);
+          ++c_lane;
+        }
+        key[32 * m + lane] = kv;
+        gm[g] = max(gm[g], kv);
+      }
+    }
+    __syncwarp();
+    const int c = __reduce_add_sync(0xffffffffu, c_lane);
+    const int k = row_budget(a, b, hs, i, c);
+    if (lane == 0 && k < c && a.not_covered && *reinterpret_cast<volatile unsigned int *>(a.not_covered) == 0u)
+      atomicOr(a.not_covered, 1u);
+    uint32_t T = 0xFFFFFFFFu;
+    int take = 0;
+    if (k >= c) {
+      T = 0u;
+    } else if (k > 0) {
+      bool done = false;
+      if (k <= 32 * GPL) {
+        const uint32_t L = warp_kth_largest<GPL>(gm, k);
+        int n = 0;
+#pragma unroll 8
+        for (int m = 0; m < KPL; ++m) {
+          const uint32_t kv = key[32 * m + lane];
+          n += (kv != 0u && kv >= L) ? 1 : 0;
+        }
+        int cnt;
+        int pos = warp_excl_scan(n, lane, &cnt);
+        if (cnt <= kSelBuf) {
+#pragma unroll 8
+          for (int m = 0; m < KPL; ++m) {
+            const uint32_t kv = key[32 * m + lane];
+            if (kv != 0u && kv >= L) buf[pos++] = kv;
+          }
+          __syncwarp();
+          if (cnt <= 128) {
+            uint32_t y[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int q = lane * 4 + e;
+              y[e] = q < cnt ? buf[q] : 0u;
+            }
+            __syncwarp();
+            T = warp_kth_largest<4>(y, k);
+          } else {
+            uint32_t y[kSelBuf / 32];
+#pragma unroll
+            for (int e = 0; e < kSelBuf / 32; ++e) {
+              const int q = lane * (kSelBuf / 32) + e;
+              y[e] = q < cnt ? buf[q] : 0u;
+            }
+            __syncwarp();
+            T = warp_kth_largest<kSelBuf / 32>(y, k);
+          }
+          done = true;
+        }
+      }
+      if (!done) T = warp_kth_range_smem(key, 32 * KPL, k, buf);
+      int above = 0;
+#pragma unroll 8
+      for (int m = 0; m < KPL; ++m) {
+        const uint32_t kv = key[32 * m + lane];
+        above += (kv != 0u && kv > T) ? 1 : 0;
+      }
+      take = k - __reduce_add_sync(0xffffffffu, above);
+    }
+    // lane l's span: tiles 64 l .. 64 l + 63, i.e. entries 64 l + r of the
+    // tile-ordered keys; flags for > T (or every candidate), forced, ties
+    const int span0 = 64 * lane;
+    uint32_t gt[2] = {0u, 0u}, tw[2] = {0u, 0u};
+    if (span0 < 32 * KPL) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll 8
+        for (int r = 0; r < 32; ++r) {
+          const int j = span0 + 32 * h + r;
+          const uint32_t kv = key[j];
+          const bool forced = j < NK && is_forced(j);
+          if ((kv != 0u && (kv > T || k >= c)) || forced) gt[h] |= 1u << r;
+          if (take > 0 && kv != 0u && kv == T) tw[h] |= 1u << r;
+        }
+    }
+    __syncwarp();  // every lane has read the keys before the warp's next row
+    // the first `take` ties in tile order join the keep
+    int tie_tot;
+    const int tie_before = warp_excl_scan(__popc(tw[0]) + __popc(tw[1]), lane, &tie_tot);
+    int room = take - tie_before;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t w = tw[h];
+      while (w != 0u && room > 0) {
+        const uint32_t bit = w & (0u - w);
+        gt[h] |= bit;
+        w ^= bit;
+        --room;
+      }
+    }
+    int kept_tot;
+    int pos = warp_excl_scan(__popc(gt[0]) + __popc(gt[1]), lane, &kept_tot);
+    int8_t *krow = a.keep ? a.keep + row * NK : nullptr;
+    uint16_t *irow = a.kv_index ? a.kv_index + row * NK : nullptr;
+    if (krow && span0 < NK) {
+      if (keep16 && span0 + 64 <= NK) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int qq = 0; qq < 2; ++qq) {
+            uint32_t wd[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const uint32_t nib = (gt[h] >> (16 * qq + 4 * u)) & 0xFu;
+              wd[u] = (nib & 1u) | ((nib >> 1) & 1u) << 8 | ((nib >> 2) & 1u) << 16 | ((nib >> 3) & 1u) << 24;
+            }
+            *reinterpret_cast<uint4 *>(krow + span0 + 32 * h + 16 * qq) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+          }
+      } else {
+        for (int r = 0; r < 64 && span0 + r < NK; ++r) krow[span0 + r] = (int8_t)((gt[r >> 5] >> (r & 31)) & 1u);
+      }
+    }
+    if (irow) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t w = gt[h];
+        while (w != 0u) {
+          const int r = __ffs(w) - 1;
+          w &= w - 1u;
+          irow[pos++] = (uint16_t)(span0 + 32 * h + r);
+        }
+      }
+    }
+    if (lane == 0 && a.kv_count) a.kv_count[row] = kept_tot;
+  }
 }
 
 // ----------------------------------------------------------------- chunked
@@ -996,6 +1263,11 @@ cudaError_t launch_k(K kernel, dim3 grid, size_t smem, const SelectArgs &a, cuda
   return launch_pdl(kernel, grid, dim3(kThreads), smem, stream, a);
 }
 
+template <typename K>
+cudaError_t launch_sel(K kernel, dim3 grid, const SelectArgs &a, cudaStream_t stream) {
+  return launch_pdl(kernel, grid, dim3(kSelWarps * 32), 0, stream, a);
+}
+
 // Cooperative launch: every CTA of the grid is resident at once (the launch
 // fails otherwise), which the in-kernel group wait relies on.
 template <typename K>
@@ -1072,18 +1344,16 @@ cudaError_t launch_select(const SelectArgs &a, int num_sms, cudaStream_t stream)
                      : launch_k(select_fusedq_kernel<128>, grid, smem, a, stream);
   }
   if (a.tc_scores != nullptr && a.scores_out == nullptr && select_uses_tc_scores(a.NK, a.D, a.head_shared)) {
-    // scores on the tensor cores into the scratch, then the top-k from there
-    const ScoreTcArgs st = {a.pq, a.pk, a.B, a.Hs, a.Hkv, a.NQ, a.NK, round_up(a.NK, 128), a.D, 1, a.tc_scores,
-                            a.err};
-    cudaError_t e = launch_score_tc(st, num_sms, stream);
-    if (e != cudaSuccess) return e;
-    const dim3 grid((a.NQ + 7) / 8, a.Hs, a.B);
+    // the scores are in the scratch (launch_score_tc ran before): top-k
     const int nkp = round_up(a.NK, 128);
-    if (nkp <= 128) return launch_k(select_scores_kernel<4>, grid, 0, a, stream);
-    if (nkp <= 256) return launch_k(select_scores_kernel<8>, grid, 0, a, stream);
-    if (nkp <= 512) return launch_k(select_scores_kernel<16>, grid, 0, a, stream);
-    if (nkp <= 1024) return launch_k(select_scores_kernel<32>, grid, 0, a, stream);
-    return launch_k(select_scores_kernel<64>, grid, 0, a, stream);
+    const long long rows = (long long)a.B * a.Hs * a.NQ;
+    // one warp per row, rows taken in turn by the resident CTAs
+    const dim3 g1((unsigned)std::min<long long>((rows + kSelWarps - 1) / kSelWarps, (long long)num_sms * 12));
+    if (nkp <= 128) return launch_sel(select_scores_kernel<4>, g1, a, stream);
+    if (nkp <= 256) return launch_sel(select_scores_kernel<8>, g1, a, stream);
+    if (nkp <= 512) return launch_sel(select_scores_kernel<16>, g1, a, stream);
+    if (nkp <= 1024) return launch_sel(select_scores_kernel<32>, g1, a, stream);
+    return launch_sel(select_scores_kernel<64>, g1, a, stream);
   }
   const int R = select_rows_per_cta(a.B, a.Hs, a.NQ, a.NK, num_sms, a.D, a.head_shared);
   if (R == 0) return cudaErrorInvalidValue;

@@ -130,6 +130,10 @@ _W += [
              budget=0.15, pins_drops="sinks2_blockcausal"),
     Workload("long_kv_hs", B=1, Hq=4, Hkv=2, Sq=512, Skv=16384, D=128,
              budget=0.10, head_shared=True),
+    # rows of 2048 kv tiles, as in the Large-2D workload (the longest rows
+    # the register top-k holds), at a size the oracle selects in full
+    Workload("long_kv_2k", B=1, Hq=2, Hkv=1, Sq=1024, Skv=131072, D=64,
+             budget=0.05),
     # one kv group of the Large 2D-local workload (8 query heads, 1/8 of its
     # work), for profiling captures that must stay small; per kv group the
     # kernels see the same shapes, statistics and schedule
