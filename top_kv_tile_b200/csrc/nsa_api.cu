@@ -318,8 +318,9 @@ nsa_status run_tc_scores(const float *pq, const float *pk, int B, int Hq, int Hk
   NSA_CUDA(nsa::launch_split_tf32(pk, (long long)B * Hkv * NK * D, hi, lo, dev->num_sms, s));
   CUtensorMap thi, tlo;
   nsa_status st;
-  if ((st = encode_f32_rows(&thi, hi, D, NK, (long long)B * Hkv, 256)) != NSA_OK) return st;
-  if ((st = encode_f32_rows(&tlo, lo, D, NK, (long long)B * Hkv, 256)) != NSA_OK) return st;
+  const int rows = nsa::score_tc_chunk(B, Hq, NQ, NK, dev->num_sms);
+  if ((st = encode_f32_rows(&thi, hi, D, NK, (long long)B * Hkv, rows)) != NSA_OK) return st;
+  if ((st = encode_f32_rows(&tlo, lo, D, NK, (long long)B * Hkv, rows)) != NSA_OK) return st;
   const nsa::ScoreTcArgs a = {pq, pk, B, Hq, Hkv, NQ, NK, (int)cdiv(NK, 128) * 128, D, 1, scores, dev->err};
   NSA_CUDA(nsa::launch_score_tc(a, thi, tlo, dev->num_sms, s));
   return NSA_OK;

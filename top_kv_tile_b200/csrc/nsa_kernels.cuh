@@ -101,8 +101,8 @@ struct SelectArgs {
 // = pq (B, Hq, NQ, D) . pk (B, Hkv, NK, D)^T, query head h against kv head
 // h / (Hq / Hkv); columns from NK up to NKP hold zeros. The keys come as
 // their tf32 hi and lo parts (launch_split_tf32), read through the tensor
-// maps thi / tlo: {D, NK, B*Hkv} float32, boxes {32, 256, 1}, 128-byte
-// swizzle.
+// maps thi / tlo: {D, NK, B*Hkv} float32, boxes {32, score_tc_chunk(..), 1},
+// 128-byte swizzle.
 struct ScoreTcArgs {
   const float *pq;
   const float *pk;
@@ -113,6 +113,9 @@ struct ScoreTcArgs {
 };
 cudaError_t launch_score_tc(ScoreTcArgs a, const CUtensorMap &thi, const CUtensorMap &tlo, int num_sms,
                             cudaStream_t stream);
+// The kv tiles per chunk (the MMA's N, 256 or 64) launch_score_tc uses for
+// these sizes; the tensor maps' boxes must have that many rows.
+int score_tc_chunk(int B, int Hq, int NQ, int NK, int num_sms);
 size_t score_tc_smem(int D);
 // hi = tf32(x), lo = tf32(x - hi) elementwise (n a multiple of 4, 16-byte
 // aligned arrays).

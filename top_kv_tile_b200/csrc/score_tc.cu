@@ -18,9 +18,10 @@
 // whole shared memory holds key tiles. The keys stream in by TMA in chunks
 // of 256 kv tiles (N = 256: one MMA instruction does four times the work of
 // an N = 64 one, and issuing MMAs, not executing them, is what bounds a
-// single issuing thread), one 32-element segment of the head dimension (hi
-// and lo, 64 KB) per ring stage. Per segment 4 K-steps x 3 products go into
-// a 256-column f32 accumulator in TMEM; the epilogue warps (one query row
+// single issuing thread; chunks of 64 when 256-wide ones would leave SMs
+// idle), one 32-element segment of the head dimension (hi and lo) per ring
+// stage. Per segment 4 K-steps x 3 products go into an N-column f32
+// accumulator in TMEM; the epilogue warps (one query row
 // per thread) copy each finished chunk to the score scratch and free the
 // accumulator for the next chunk. Every wait is bounded.
 #include <algorithm>
@@ -32,16 +33,21 @@ namespace nsa {
 
 namespace {
 
-constexpr int TM = 128;                          // query rows per CTA (the MMA's M)
-constexpr int TN = 256;                          // kv tiles per chunk (the MMA's N)
-constexpr int KSEG = 32;                         // f32 elements of D per 128-byte row
-constexpr int KST = 3;                           // ring stages
-constexpr int SEG_BYTES = TN * 128;              // one D segment of a chunk, hi or lo (32 KB)
-constexpr int STAGE_BYTES = 2 * SEG_BYTES;       // hi, then lo
-constexpr int OFF_BAR = KST * STAGE_BYTES;       // 192 KB of key tiles
-constexpr int TILE_BYTES = OFF_BAR + 256;
-constexpr int kTcThreads = 192;                  // 6 warps
+constexpr int TM = 128;   // query rows per CTA (the MMA's M)
+constexpr int KSEG = 32;  // f32 elements of D per 128-byte row
+constexpr int KST = 3;    // ring stages
+constexpr int kTcThreads = 192;  // 6 warps
 constexpr uint32_t COL_QHI = 0, COL_QLO = 128, COL_ACC = 256, TMEM_COLS = 512;
+
+// TN kv tiles per chunk (the MMA's N): 256 normally; 64 when the grid would
+// otherwise not cover the SMs (a few row blocks and short rows).
+template <int TN>
+struct TcCfg {
+  static constexpr int SEG_BYTES = TN * 128;         // one D segment of a chunk, hi or lo
+  static constexpr int STAGE_BYTES = 2 * SEG_BYTES;  // hi, then lo
+  static constexpr int OFF_BAR = KST * STAGE_BYTES;
+  static constexpr int TILE_BYTES = OFF_BAR + 256;
+};
 
 struct TcBars {
   uint64_t full[KST];
@@ -81,11 +87,13 @@ __global__ void split_tf32_kernel(const float4 *x, long long n4, float4 *hi, flo
   }
 }
 
-template <int D>
+template <int D, int TN>
 __global__ void __launch_bounds__(kTcThreads, 1)
     score_tc_kernel(const ScoreTcArgs a, const __grid_constant__ CUtensorMap thi,
                     const __grid_constant__ CUtensorMap tlo) {
   constexpr int NSEG = D / KSEG;
+  constexpr int SEG_BYTES = TcCfg<TN>::SEG_BYTES, STAGE_BYTES = TcCfg<TN>::STAGE_BYTES;
+  constexpr int OFF_BAR = TcCfg<TN>::OFF_BAR, TILE_BYTES = TcCfg<TN>::TILE_BYTES;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_u32 & 1023u)) & 1023u;
@@ -250,7 +258,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 size_t score_tc_smem(int D) {
   (void)D;
-  return (size_t)TILE_BYTES;
+  return (size_t)TcCfg<256>::TILE_BYTES;
 }
 
 cudaError_t launch_split_tf32(const float *x, long long n, float *hi, float *lo, int num_sms, cudaStream_t stream) {
@@ -263,26 +271,39 @@ cudaError_t launch_split_tf32(const float *x, long long n, float *hi, float *lo,
                     reinterpret_cast<float4 *>(lo));
 }
 
-cudaError_t launch_score_tc(ScoreTcArgs a, const CUtensorMap &thi, const CUtensorMap &tlo, int num_sms,
-                            cudaStream_t stream) {
+namespace {
+
+template <int D, int TN>
+cudaError_t launch_tc_t(ScoreTcArgs a, const CUtensorMap &thi, const CUtensorMap &tlo, int num_sms,
+                        cudaStream_t stream) {
   const int nchunks = (a.NK + TN - 1) / TN;
   const long long blocks = (long long)((a.NQ + TM - 1) / TM) * a.Hq * a.B;
   if (blocks == 0 || nchunks == 0) return cudaSuccess;
   // few row blocks: split the kv range so the grid covers the device
   a.nsplit = (int)std::min<long long>(nchunks, std::max<long long>(1, (num_sms + blocks - 1) / blocks));
   const dim3 grid((unsigned)((a.NQ + TM - 1) / TM), (unsigned)a.Hq, (unsigned)(a.B * a.nsplit));
-  const int smem = TILE_BYTES;
-  cudaError_t e;
-  if (a.D == 64) {
-    if ((e = cudaFuncSetAttribute(score_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
-        cudaSuccess)
-      return e;
-    return launch_pdl(score_tc_kernel<64>, grid, dim3(kTcThreads), (size_t)smem, stream, a, thi, tlo);
-  }
-  if ((e = cudaFuncSetAttribute(score_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
-      cudaSuccess)
-    return e;
-  return launch_pdl(score_tc_kernel<128>, grid, dim3(kTcThreads), (size_t)smem, stream, a, thi, tlo);
+  const int smem = TcCfg<TN>::TILE_BYTES;
+  cudaError_t e =
+      cudaFuncSetAttribute(score_tc_kernel<D, TN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(score_tc_kernel<D, TN>, grid, dim3(kTcThreads), (size_t)smem, stream, a, thi, tlo);
+}
+
+}  // namespace
+
+int score_tc_chunk(int B, int Hq, int NQ, int NK, int num_sms) {
+  // N = 256 when row blocks x 256-wide chunks cover the SMs, else N = 64
+  const long long blocks = (long long)((NQ + TM - 1) / TM) * Hq * B;
+  return blocks * ((NK + 255) / 256) >= num_sms ? 256 : 64;
+}
+
+cudaError_t launch_score_tc(ScoreTcArgs a, const CUtensorMap &thi, const CUtensorMap &tlo, int num_sms,
+                            cudaStream_t stream) {
+  const bool wide = score_tc_chunk(a.B, a.Hq, a.NQ, a.NK, num_sms) == 256;
+  if (a.D == 64)
+    return wide ? launch_tc_t<64, 256>(a, thi, tlo, num_sms, stream) : launch_tc_t<64, 64>(a, thi, tlo, num_sms, stream);
+  return wide ? launch_tc_t<128, 256>(a, thi, tlo, num_sms, stream)
+              : launch_tc_t<128, 64>(a, thi, tlo, num_sms, stream);
 }
 
 }  // namespace nsa
