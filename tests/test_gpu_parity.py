@@ -239,3 +239,56 @@ def test_tensor_core_scores_within_split_precision_bound(nsa, name, seed):
     assert np.all(err <= 2.0 ** -18 * mag + 1e-30), float((err / mag).max())
     # far below the 2^-11 relative error of a single tf32 product
     assert (err / mag).max() < 2.0 ** -19
+
+
+def _pair_keep_patterns(wl, seed):
+    """Keep tensors whose neighbouring heads keep very different tiles: long
+    runs kept by one head only, one head keeping nothing, identical lists,
+    and independent random lists (rows cycle through the patterns)."""
+    rng = np.random.default_rng(seed)
+    keep = np.zeros((wl.B, wl.Hs, wl.NQ, wl.NK), dtype=np.int8)
+    nk = wl.NK
+    for b in range(wl.B):
+        for hp in range(0, wl.Hq, 2):
+            for i in range(wl.NQ):
+                kind = (b * wl.Hq + hp + i) % 5
+                a0 = np.zeros(nk, dtype=bool)
+                a1 = np.zeros(nk, dtype=bool)
+                if kind == 0:    # runs of 1..17 tiles alternating between the heads
+                    j, cur = 0, 0
+                    while j < nk:
+                        r = int(rng.integers(1, 18))
+                        (a0 if cur == 0 else a1)[j:j + r] = True
+                        j += r
+                        cur ^= 1
+                elif kind == 1:  # head 0 keeps the first and last tiles, head 1 all between
+                    a0[0] = a0[nk - 1] = True
+                    a1[1:nk - 1] = True
+                elif kind == 2:  # one head keeps nothing
+                    a1[rng.random(nk) < 0.4] = True
+                elif kind == 3:  # identical lists
+                    a0[rng.random(nk) < 0.3] = True
+                    a1[:] = a0
+                else:            # independent
+                    a0[rng.random(nk) < 0.2] = True
+                    a1[rng.random(nk) < 0.5] = True
+                keep[b, hp, i] = a0
+                keep[b, hp + 1, i] = a1
+    return keep
+
+
+@pytest.mark.parametrize("name", ["long_kv_small", "long_kv_ragged"])
+def test_attention_keep_patterns(nsa, name):
+    # hand-made keep rows: long runs, empty rows, identical and independent
+    # lists for the heads of a kv group, rows keeping nearly every tile
+    wl = workloads.get(name)
+    assert (wl.Hq // wl.Hkv) % 2 == 0 and not wl.head_shared
+    inp = workloads.make_inputs(wl)
+    d = _dev(inp)
+    keep = _pair_keep_patterns(wl, seed=7)
+    out, lse = nsa.nsa_block_sparse_attn_fwd(d["q"], d["k"], d["v"], torch.from_numpy(keep).cuda(), wl.scale)
+    torch.cuda.synchronize()
+    nsa.nsa_device_status()
+    q, k, v = (inp[x].double().numpy() for x in "qkv")
+    ro, rl = oracle.block_sparse_attention(q, k, v, keep, wl.block_q, wl.block_kv, wl.scale)
+    parity.check_attention(out.float().cpu().numpy(), lse.cpu().numpy(), ro, rl)
