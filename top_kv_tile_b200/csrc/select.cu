@@ -922,8 +922,8 @@ __device__ __noinline__ uint32_t warp_kth_range_smem(const uint32_t *key, int n,
 
 template <int KPL>
 __global__ void __launch_bounds__(kSelWarps * 32, 6) select_scores_kernel(SelectArgs a) {
-  __shared__ uint32_t skey[kSelWarps][32 * KPL];
-  __shared__ uint32_t sbuf[kSelWarps][kSelBuf];
+  __shared__ __align__(16) uint32_t skey[kSelWarps][32 * KPL];
+  __shared__ __align__(16) uint32_t sbuf[kSelWarps][kSelBuf];
   pdl_wait();  // the scores come from the previous kernel
   const int NK = a.NK, NQ = a.NQ;
   const int NKP = round_up(NK, 128);
@@ -1003,24 +1003,36 @@ __global__ void __launch_bounds__(kSelWarps * 32, 6) select_scores_kernel(Select
             if (kv != 0u && kv >= L) buf[pos++] = kv;
           }
           __syncwarp();
+          // lane l takes entries N l .. N l + N - 1 as 16-byte loads (no
+          // bank conflicts); entries past cnt count as 0
           if (cnt <= 128) {
             uint32_t y[4];
+            const uint4 v = *reinterpret_cast<const uint4 *>(buf + lane * 4);
+            y[0] = v.x;
+            y[1] = v.y;
+            y[2] = v.z;
+            y[3] = v.w;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int q = lane * 4 + e;
-              y[e] = q < cnt ? buf[q] : 0u;
-            }
+            for (int e = 0; e < 4; ++e)
+              if (lane * 4 + e >= cnt) y[e] = 0u;
             __syncwarp();
             T = warp_kth_largest<4>(y, k);
           } else {
-            uint32_t y[kSelBuf / 32];
+            constexpr int NB = kSelBuf / 32;
+            uint32_t y[NB];
 #pragma unroll
-            for (int e = 0; e < kSelBuf / 32; ++e) {
-              const int q = lane * (kSelBuf / 32) + e;
-              y[e] = q < cnt ? buf[q] : 0u;
+            for (int e4 = 0; e4 < NB / 4; ++e4) {
+              const uint4 v = *reinterpret_cast<const uint4 *>(buf + lane * NB + 4 * e4);
+              y[4 * e4] = v.x;
+              y[4 * e4 + 1] = v.y;
+              y[4 * e4 + 2] = v.z;
+              y[4 * e4 + 3] = v.w;
             }
+#pragma unroll
+            for (int e = 0; e < NB; ++e)
+              if (lane * NB + e >= cnt) y[e] = 0u;
             __syncwarp();
-            T = warp_kth_largest<kSelBuf / 32>(y, k);
+            T = warp_kth_largest<NB>(y, k);
           }
           done = true;
         }
@@ -1034,21 +1046,27 @@ __global__ void __launch_bounds__(kSelWarps * 32, 6) select_scores_kernel(Select
       }
       take = k - __reduce_add_sync(0xffffffffu, above);
     }
-    // lane l's span: tiles 64 l .. 64 l + 63, i.e. entries 64 l + r of the
-    // tile-ordered keys; flags for > T (or every candidate), forced, ties
+    // lane l's span: tiles 64 l .. 64 l + 63, as two flag words (> T or
+    // every candidate, or forced; ties). The flags are read in the key
+    // layout (tile 32 m + lane, conflict-free) and the ballot over column
+    // block m is the flag word of tiles 32 m .. 32 m + 31: word m & 1 of
+    // lane m / 2's span
     const int span0 = 64 * lane;
     uint32_t gt[2] = {0u, 0u}, tw[2] = {0u, 0u};
-    if (span0 < 32 * KPL) {
+#pragma unroll 4
+    for (int m2 = 0; m2 < KPL / 2; ++m2) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
-#pragma unroll 8
-        for (int r = 0; r < 32; ++r) {
-          const int j = span0 + 32 * h + r;
-          const uint32_t kv = key[j];
-          const bool forced = j < NK && is_forced(j);
-          if ((kv != 0u && (kv > T || k >= c)) || forced) gt[h] |= 1u << r;
-          if (take > 0 && kv != 0u && kv == T) tw[h] |= 1u << r;
+      for (int h = 0; h < 2; ++h) {
+        const int j = 64 * m2 + 32 * h + lane;
+        const uint32_t kv = key[j];
+        const bool forced = j < NK && is_forced(j);
+        const uint32_t bg = __ballot_sync(0xffffffffu, (kv != 0u && (kv > T || k >= c)) || forced);
+        const uint32_t bt = __ballot_sync(0xffffffffu, take > 0 && kv != 0u && kv == T);
+        if (lane == m2) {
+          gt[h] = bg;
+          tw[h] = bt;
         }
+      }
     }
     __syncwarp();  // every lane has read the keys before the warp's next row
     // the first `take` ties in tile order join the keep
