@@ -120,16 +120,29 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int g = a.Hq / a.Hkv;
 
-  // work item: consecutive CTAs share a kv head (L2 reuse of K and V)
+  // work item: query tiles in descending order, so that where the kept
+  // count grows with the tile index (a drop rule forbidding the future) the
+  // long rows start first. Consecutive CTAs are the query heads of one kv
+  // group. With q_first the query tile is the slowest index: the longest
+  // rows of every head and batch start in the first wave and the short
+  // ones fill the last (grids of few waves, where the tail counts).
+  // Otherwise the query tile comes next after the head in the group, so
+  // the resident CTAs share one kv head's K and V in L2.
   long long x = blockIdx.x;
   const int hh = (int)(x % g);
   x /= g;
-  // query tiles in descending order: where the kept count grows with the
-  // tile index (a drop rule forbidding the future) the long rows start first
-  const int i = a.NQ - 1 - (int)(x % a.NQ);
-  x /= a.NQ;
-  const int hk = (int)(x % a.Hkv);
-  const int b = (int)(x / a.Hkv);
+  int i, hk, b;
+  if (a.q_first) {
+    hk = (int)(x % a.Hkv);
+    x /= a.Hkv;
+    b = (int)(x % a.B);
+    i = a.NQ - 1 - (int)(x / a.B);
+  } else {
+    i = a.NQ - 1 - (int)(x % a.NQ);
+    x /= a.NQ;
+    hk = (int)(x % a.Hkv);
+    b = (int)(x / a.Hkv);
+  }
   const int h = hk * g + hh;
 
   if (threadIdx.x == 0) {
@@ -473,8 +486,11 @@ cudaError_t launch_attn_fwd(const AttnArgs &a, int D, const CUtensorMap &tq, con
 
 cudaError_t launch_attn_fwd(const AttnArgs &a, int D, int num_sms, const CUtensorMap &tq, const CUtensorMap &tk,
                             const CUtensorMap &tv, cudaStream_t stream) {
-  (void)num_sms;
-  return launch_attn_fwd(a, D, tq, tk, tv, stream);
+  // query-tile-first order for grids of at most 16 waves (two CTAs per SM)
+  AttnArgs b = a;
+  const long long ctas = (long long)a.B * a.Hq * a.NQ;
+  b.q_first = ctas <= 16LL * 2 * num_sms ? 1 : 0;
+  return launch_attn_fwd(b, D, tq, tk, tv, stream);
 }
 
 }  // namespace nsa

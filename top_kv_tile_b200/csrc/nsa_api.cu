@@ -298,6 +298,7 @@ nsa_status run_attention(const void *q, const void *k, const void *v, const Geom
   a.lse = lse;
   a.err = dev->err;
   a.kmask = kmask;
+  a.q_first = 0;  // chosen by the launcher
   for (int d = 0; d < 3; ++d) a.ks[d] = 0;
   if (kmask) {
     a.ks[0] = kmask_strides ? kmask_strides[0] : (long long)g.Hkv * g.Skv;

@@ -185,6 +185,8 @@ struct AttnArgs {
   // whose byte is 0 takes part in no query row of that kv head (null = none)
   const int8_t *kmask;
   long long ks[3];
+  // CTA order: 1 = query tile slowest (set by the launcher from the grid size)
+  int q_first;
 };
 
 cudaError_t launch_attn_fwd(const AttnArgs &a, int D, int num_sms, const CUtensorMap &tq, const CUtensorMap &tk,
