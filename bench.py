@@ -526,17 +526,26 @@ def headline_extras(nsa, wl, inp, q, k, v, pins, drops, spec, keep, out, lse, ws
     ho = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
     hl = [torch.empty(lse.shape, dtype=lse.dtype).pin_memory() for _ in range(2)]
     e0, e1 = _ev(), _ev()
+    ec = [_ev() for _ in range(4)]  # around the copies of the first timed step
     for it in range(1 + e2e_steps):
         if it == 1:
             barrier(world, dev)
             torch.cuda.synchronize()
             e0.record()
+        if it == 1:
+            ec[0].record()
         q.copy_(hq, non_blocking=True)
         k.copy_(hk_, non_blocking=True)
         v.copy_(hv, non_blocking=True)
+        if it == 1:
+            ec[1].record()
         nsa.nsa_forward(q, k, v, spec, wl.scale, pins, drops, keep_out=keep, out=out, lse=lse, ws=ws)
+        if it == 1:
+            ec[2].record()
         ho[0].copy_(out, non_blocking=True)
         hl[0].copy_(lse, non_blocking=True)
+        if it == 1:
+            ec[3].record()
     e1.record()
     torch.cuda.synchronize()
     barrier(world, dev)
@@ -592,13 +601,23 @@ def headline_extras(nsa, wl, inp, q, k, v, pins, drops, spec, keep, out, lse, ws
     e2e_ms = pipe_ms if pipe_ok else serial_ms
     h2d = sum(t.numel() * t.element_size() for t in (q, k, v))
     d2h = ho[0].numel() * ho[0].element_size() + hl[0].numel() * hl[0].element_size()
+    # the link's own rates, from the copies of one serial step (each alone on
+    # the link): with copy-in and copy-out overlapped, a step cannot take
+    # less than the longer of the two
+    h2d_gbs = h2d / (ec[0].elapsed_time(ec[1]) * 1e-3) / 1e9
+    d2h_gbs = d2h / (ec[2].elapsed_time(ec[3]) * 1e-3) / 1e9
+    link_ms = max(h2d / h2d_gbs, d2h / d2h_gbs) / 1e6
     res["e2e"] = {
         "value": round(flops_all / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s", "ms_per_step": round(e2e_ms, 4),
         "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
         "schedule": ("copy-in, compute and copy-out on three streams, two device buffer sets" if pipe_ok
                      else "single stream"),
         "single_stream_ms_per_step": round(serial_ms, 4),
-        "single_stream_value": round(flops_all / (serial_ms * 1e-3) / 1e12, 3)}
+        "single_stream_value": round(flops_all / (serial_ms * 1e-3) / 1e12, 3),
+        "link": {"h2d_gbs": round(h2d_gbs, 2), "d2h_gbs": round(d2h_gbs, 2), "bound_ms_per_step": round(link_ms, 3),
+                 "frac": round(link_ms / e2e_ms, 4),
+                 "note": "measured on this step's own copies, each direction alone; the bound is the longer "
+                         "direction's time, the pipelined step's floor when the two directions overlap"}}
     return res
 
 
@@ -739,7 +758,7 @@ def main(argv=None):
                     help="the headline workload (default: Large 2D-local, the largest one-GPU configuration)")
     ap.add_argument("--config-steps", type=int, default=20,
                     help="timed steps for each workload of the configs block (at most --steps)")
-    ap.add_argument("--e2e-steps", type=int, default=10, help="timed end-to-end steps (at most --steps)")
+    ap.add_argument("--e2e-steps", type=int, default=20, help="timed end-to-end steps (at most --steps)")
     ap.add_argument("--cpu-seconds", type=float, default=6.0,
                     help="oracle seconds per workload for the CPU baseline (at least one unit)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
