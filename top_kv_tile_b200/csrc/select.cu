@@ -183,11 +183,13 @@ __device__ __forceinline__ uint32_t warp_kth_largest(uint32_t (&x)[N], int k) {
 // largest; a bin one key wide is the exact key. The first interval is the
 // keys' own range, from their minimum to their maximum: a row's scores share
 // their leading bits, so bins cut from the top bits of the key would pile
-// nearly every key into one bin (and its counter). Every lane returns the
-// same value.
+// nearly every key into one bin (and its counter). Once the bin that holds
+// the k-th largest has at most 32 keys, those keys are gathered and sorted
+// across the warp instead of cutting the bin further. Every lane returns
+// the same value.
 template <int G>
 __device__ __forceinline__ uint32_t warp_kth_interval(const uint32_t (&kk)[G][4], int kr, uint32_t lo, uint32_t hi) {
-  __shared__ int hist_all[kThreads / 32][256];
+  __shared__ __align__(16) int hist_all[kThreads / 32][256];
   int *hist = hist_all[threadIdx.x / 32];
   const int lane = threadIdx.x & 31;
 #pragma unroll 1
@@ -204,13 +206,23 @@ __device__ __forceinline__ uint32_t warp_kth_interval(const uint32_t (&kk)[G][4]
         if (key >= lo && key <= hi) atomicAdd(&hist[(key - lo) >> shift], 1);
       }
     __syncwarp();
-    // lane l holds bins 255 - 8 l down to 248 - 8 l (descending)
+    // lane l holds bins 255 - 8 l down to 248 - 8 l (descending), read as two
+    // 16-byte vectors (bins 248 - 8 l .. 255 - 8 l)
     int c8[8], sum = 0;
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      c8[q] = hist[255 - (lane * 8 + q)];
-      sum += c8[q];
+    {
+      const int4 b0 = *reinterpret_cast<const int4 *>(hist + 248 - 8 * lane);
+      const int4 b1 = *reinterpret_cast<const int4 *>(hist + 252 - 8 * lane);
+      c8[0] = b1.w;
+      c8[1] = b1.z;
+      c8[2] = b1.y;
+      c8[3] = b1.x;
+      c8[4] = b0.w;
+      c8[5] = b0.z;
+      c8[6] = b0.y;
+      c8[7] = b0.x;
     }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) sum += c8[q];
     int incl = sum;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -219,12 +231,13 @@ __device__ __forceinline__ uint32_t warp_kth_interval(const uint32_t (&kk)[G][4]
     }
     const int excl = incl - sum;  // keys of the interval in higher bins than this lane's
     const bool mine = excl < kr && kr <= incl;
-    int bin = 0, above = excl;
+    int bin = 0, above = excl, cb = 0;
     if (mine) {
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         if (above + c8[q] >= kr) {
           bin = 255 - (lane * 8 + q);
+          cb = c8[q];
           break;
         }
         above += c8[q];
@@ -233,12 +246,33 @@ __device__ __forceinline__ uint32_t warp_kth_interval(const uint32_t (&kk)[G][4]
     const int src = __ffs(__ballot_sync(0xffffffffu, mine)) - 1;
     bin = __shfl_sync(0xffffffffu, bin, src);
     above = __shfl_sync(0xffffffffu, above, src);
+    cb = __shfl_sync(0xffffffffu, cb, src);
     kr -= above;
     const uint32_t nlo = lo + ((uint32_t)bin << shift);
     const uint32_t width = (1u << shift) - 1u;
     hi = (hi - nlo < width) ? hi : nlo + width;
     lo = nlo;
-    __syncwarp();  // every lane has read the histogram before it is cleared
+    __syncwarp();  // every lane has read the histogram before it is reused
+    if (cb <= 32 && lo < hi) {
+      // the bin's keys (at most 32) into the histogram's space, one per lane,
+      // then the kr-th largest of them (the zero padding sorts below them)
+      int n_in = 0;
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) n_in += (kk[g][e] >= lo && kk[g][e] <= hi) ? 1 : 0;
+      int tot;
+      int pos = warp_excl_scan(n_in, lane, &tot);
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (kk[g][e] >= lo && kk[g][e] <= hi) hist[pos++] = (int)kk[g][e];
+      __syncwarp();
+      uint32_t x[1] = {lane < tot ? (uint32_t)hist[lane] : 0u};
+      __syncwarp();  // every lane has read its key before the histogram is reused
+      return warp_kth_largest<1>(x, kr);
+    }
   }
   return lo;
 }
