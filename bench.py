@@ -17,7 +17,9 @@ The headline workload is the largest one-GPU configuration, Large 2D-local
   (q + k read, keep written, pin/drop masks read, timed as one span from
   before pooling to after selection so its kernels overlap as in a step),
   each also as a fraction of the measured peaks; roofline: the attention
-  kernel against the bf16 tensor peak;
+  kernel against the bf16 tensor peak: the sustained one (a GEMM held under
+  the power cap) when the power cap was active during the timed steps, else
+  the burst one, with the fraction of the burst peak always beside it;
 - e2e: the same metric through nsa_forward from pinned host buffers, every
   step copying q, k, v in and O, LSE out (copy-in, compute and copy-out on
   three streams over two device buffer sets; the single-stream figure is
@@ -662,6 +664,21 @@ def run_ours(args):
         return
     wl = head["wl"]
     cpu = head["summary"].get("cpu_baseline")
+    # the tensor peak paired with how the kernel ran: the sustained figure
+    # (a GEMM held for seconds under the 1 kW power cap) when the power cap
+    # was active during the timed steps, else the burst figure; the fraction
+    # of the burst peak is kept beside it either way
+    clk = head["clocks"] or {}
+    capped = "sw_power_cap" in (clk.get("reasons") or [])
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peak_t))
+    roof_peak = peak_sus if capped else peak_t
+    roofline = {
+        "kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": round(head["attn_tflops"], 2),
+        "peak": roof_peak, "unit": "TFLOP/s", "frac": round(head["attn_tflops"] / roof_peak, 4),
+        "peak_source": (f"{peak_src} bf16_tflops_sustained (sw_power_cap active during the timed steps)" if capped
+                        else f"{peak_src} bf16_tflops (burst)"),
+        "frac_of_burst": round(head["attn_tflops"] / peak_t, 4), "burst_peak": peak_t,
+        "traffic": load_traffic(wl.name)}
     line = {
         "metric": METRIC,
         "value": round(head["value"], 3),
@@ -685,9 +702,7 @@ def run_ours(args):
         "selection": {"gbs": round(head["sel_gbs"], 1), "ms": round(head["sel_ms"], 5), "bytes": head["sel_bytes"],
                       "frac_hbm": round(head["sel_gbs"] / float(peaks["hbm_gbs"]), 4),
                       "pool_ms": round(head["pool_ms"], 5), "select_ms": round(head["select_ms"], 5)},
-        "roofline": {"kernel": "attn_fwd_kernel", "bound": "tensor", "achieved": round(head["attn_tflops"], 2),
-                     "peak": peak_t, "unit": "TFLOP/s", "frac": round(head["attn_tflops"] / peak_t, 4),
-                     "peak_source": f"{peak_src} bf16_tflops (burst)", "traffic": load_traffic(wl.name)},
+        "roofline": roofline,
         "e2e": head["e2e"],
         "radial_control": head["radial_control"],
         "key_mask": head["key_mask"],
@@ -696,7 +711,8 @@ def run_ours(args):
         "gpu_launches": head["launches"],
         "clocks": head["clocks"],
         "configs": configs,
-        "peaks": {"hbm_gbs": float(peaks["hbm_gbs"]), "bf16_tflops": peak_t, "source": peak_src},
+        "peaks": {"hbm_gbs": float(peaks["hbm_gbs"]), "bf16_tflops": peak_t, "bf16_tflops_sustained": peak_sus,
+                  "source": peak_src},
     }
     print(json.dumps(line), flush=True)
 
