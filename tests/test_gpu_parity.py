@@ -292,3 +292,31 @@ def test_attention_keep_patterns(nsa, name):
     q, k, v = (inp[x].double().numpy() for x in "qkv")
     ro, rl = oracle.block_sparse_attention(q, k, v, keep, wl.block_q, wl.block_kv, wl.scale)
     parity.check_attention(out.float().cpu().numpy(), lse.cpu().numpy(), ro, rl)
+
+
+def test_attention_kv_index_beyond_int16(nsa):
+    # kept-tile indices on both sides of 2^15 (the lists are uint16) and the
+    # partial last tile of a 33,001-tile key axis; one row keeps nothing,
+    # one keeps 300 tiles, and the last query tile is partial
+    B, Hq, Hkv, D = 1, 2, 1, 64
+    Sq, NK = 3 * 128 - 57, 33001
+    Skv = (NK - 1) * 64 + 17
+    gen = torch.Generator().manual_seed(5)
+    q = torch.randn(B, Hq, Sq, D, generator=gen).to(torch.bfloat16)
+    k = torch.randn(B, Hkv, Skv, D, generator=gen).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, Skv, D, generator=gen).to(torch.bfloat16)
+    NQ = (Sq + 127) // 128
+    keep = np.zeros((B, Hq, NQ, NK), dtype=np.int8)
+    rng = np.random.default_rng(9)
+    fixed = [0, 1, 8191, 8192, 16384, 32766, 32767, 32768, 32769, NK - 2, NK - 1]
+    keep[0, 0, 0, fixed] = 1
+    keep[0, 0, 1, rng.choice(NK, 300, replace=False)] = 1
+    keep[0, 0, 2, 32768:32768 + 40] = 1
+    keep[0, 1, 0, rng.choice(np.arange(32000, NK), 25, replace=False)] = 1
+    keep[0, 1, 2, [5, NK - 1]] = 1  # row (1, 1) keeps nothing
+    out, lse = nsa.nsa_block_sparse_attn_fwd(q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(keep).cuda(), D ** -0.5)
+    torch.cuda.synchronize()
+    nsa.nsa_device_status()
+    ro, rl = oracle.block_sparse_attention(q.float().numpy(), k.float().numpy(), v.float().numpy(), keep, 128, 64,
+                                           D ** -0.5)
+    parity.check_attention(out.float().cpu().numpy(), lse.cpu().numpy(), ro, rl)
