@@ -14,7 +14,8 @@ from tests import parity
 pytestmark = pytest.mark.gpu
 
 SMALL = ["tiny", "gqa_small", "head_shared_small", "cross_small", "large2d_small",
-         "ragged", "ragged_cross", "nq1", "dense_force", "long_kv_small", "long_kv_ragged", "long_kv_hs", "long_kv_2k"]
+         "ragged", "ragged_cross", "nq1", "dense_force", "long_kv_small", "long_kv_ragged", "long_kv_hs", "long_kv_2k",
+         "long_kv_4k", "long_kv_8k_hs"]
 
 
 @pytest.fixture(scope="module")

@@ -134,6 +134,13 @@ _W += [
     # the register top-k holds), at a size the oracle selects in full
     Workload("long_kv_2k", B=1, Hq=2, Hkv=1, Sq=1024, Skv=131072, D=64,
              budget=0.05),
+    # rows past 2048 kv tiles (the scores chunked through shared memory):
+    # 4096 per head, and 8192 (the longest selection row) head-shared with a
+    # partial last kv tile
+    Workload("long_kv_4k", B=1, Hq=2, Hkv=1, Sq=512, Skv=262144, D=64,
+             budget=0.05),
+    Workload("long_kv_8k_hs", B=1, Hq=2, Hkv=2, Sq=384, Skv=524263, D=64,
+             budget=0.02, head_shared=True),
     # one kv group of the Large 2D-local workload (8 query heads, 1/8 of its
     # work), for profiling captures that must stay small; per kv group the
     # kernels see the same shapes, statistics and schedule
