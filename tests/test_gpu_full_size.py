@@ -1,5 +1,7 @@
 """GPU parity at the five workloads' full sizes, in the launch configuration
-bench.py times (nsa_forward with keep_out).
+bench.py times (nsa_forward with keep_out), and on gqa_wide, whose fused
+selection grid is larger than the device holds at once (the keys are then
+pooled by a kernel of their own).
 
 Keep rows: Tiny, GQA and Cross are checked row by row against the oracle's
 full select_blocks; Head-shared (all 256 rows) and Large2D (256 sampled rows
@@ -31,8 +33,8 @@ from tests import parity
 
 pytestmark = pytest.mark.gpu
 
-FULL = ["tiny", "gqa", "head_shared", "cross", "large2d"]
-ALL_ROWS = {"tiny", "gqa", "cross"}   # keep rows against the oracle's full selection
+FULL = ["tiny", "gqa", "head_shared", "cross", "large2d", "gqa_wide"]
+ALL_ROWS = {"tiny", "gqa", "cross", "gqa_wide"}   # keep rows against the oracle's full selection
 N_KEEP_ROWS = 256                     # sampled keep rows otherwise
 N_ATTN_TILES = 32                     # sampled attention tiles (every tile for tiny)
 
@@ -72,10 +74,17 @@ def test_full_size_from_the_oracle_keep(nsa, name):
     drops = None if inp["drops"] is None else torch.from_numpy(inp["drops"]).to(dev)
     spec = nsa.SparseSpec(wl.budget, wl.block_q, wl.block_kv, wl.head_shared, wl.force)
     keep = torch.empty(wl.B, wl.Hs, wl.NQ, wl.NK, dtype=torch.int8, device=dev)
+    n0 = nsa.nsa_kernel_launches()
     out, lse = nsa.nsa_forward(q, k, v, spec, wl.scale, pins, drops, keep_out=keep)
+    launches = nsa.nsa_kernel_launches() - n0
     torch.cuda.synchronize()
     nsa.nsa_device_status()
     gk = keep.cpu().numpy()
+    # the selection path each case is here to exercise: GQA's grid fits on
+    # the device, so one cooperative kernel pools k itself (select, then
+    # attention); gqa_wide's does not, so pool_kernel pools k first
+    if name in ("gqa", "gqa_wide"):
+        assert launches == (2 if name == "gqa" else 3), launches
 
     # every row: kept count from the plan, must-and-not-forbidden tiles present
     cnt, mf = _counts_closed_form(wl, inp["pins"], inp["drops"])
