@@ -141,7 +141,7 @@ _W += [
     # at once: the keys are then pooled by their own kernel before the select
     Workload("gqa_wide", B=8, Hq=64, Hkv=8, Sq=2048, Skv=2048, D=128,
              budget=0.30, recipe="segment_mean", params={"segment": 512, "sigma": 0.5}),
-    Workload("long_kv_4k", B=1, Hq=2, Hkv=1, Sq=512, Skv=262144, D=64,
+    Workload("long_kv_4k", B=1, Hq=2, Hkv=1, Sq=512, Skv=262144, D=128,
              budget=0.05),
     Workload("long_kv_8k_hs", B=1, Hq=2, Hkv=2, Sq=384, Skv=524263, D=64,
              budget=0.02, head_shared=True),
