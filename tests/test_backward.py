@@ -14,7 +14,7 @@ from tests import parity
 pytestmark = pytest.mark.gpu
 
 CASES = ["tiny", "gqa_small", "head_shared_small", "cross_small", "ragged", "ragged_cross", "nq1",
-         "dense_force", "large2d_small"]
+         "dense_force", "large2d_small", "long_kv_ragged", "long_kv_2k"]
 
 
 @pytest.fixture(scope="module")
