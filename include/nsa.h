@@ -216,6 +216,9 @@ size_t nsa_bwd_workspace_bytes(int B, int Hq, int Hkv, int Sq, int Skv, int D,
  * ignored, as the page's `None` asks. keep_out (nullable): when given,
  * receives the int8 keep (B,Hs,NQ,NK) of the selection (its contents are the
  * selection even when the dense short circuit is taken).
+ * The call allocates nothing and never synchronises with the host, so it can
+ * be captured into a CUDA graph; make one call on the device before the
+ * capture, which loads the module.
  * workspace: >= nsa_workspace_bytes(...) bytes, 256-byte aligned. */
 nsa_status nsa_forward(const void *q, const void *k, const void *v, int B,
                        int Hq, int Hkv, int Sq, int Skv, int D,
