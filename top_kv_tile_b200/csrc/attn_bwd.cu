@@ -119,15 +119,6 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned int *err,
-                                          unsigned int site) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err, site) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  if (ok) (void)mbar_try_wait(bar, parity);
-  return ok != 0;
-}
-
 // The key columns of kv tile j that take part, as bits (mlo: columns 0-31,
 // mhi: 32-63): inside Skv and, with a key mask, unmasked for kv head hk.
 // Called by a whole warp (the bits come from ballots).

@@ -85,18 +85,6 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
-// A whole warp waits on an mbarrier phase: lane 0 polls (bounded), then every
-// lane performs one completing try_wait so that each thread acquires the
-// phase's memory effects. Returns the same answer on every lane.
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned int *err,
-                                          unsigned int site) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err, site) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  if (ok) (void)mbar_try_wait(bar, parity);
-  return ok != 0;
-}
-
 template <int D, bool KMASK>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_fwd_kernel(const AttnArgs a, const __grid_constant__ CUtensorMap tq,

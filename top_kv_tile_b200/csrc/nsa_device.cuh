@@ -115,6 +115,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
   }
 }
 
+// A whole warp waits on an mbarrier phase. Every lane waits itself (and so
+// acquires the phase's memory effects), and the answer is made the same on
+// every lane: a lane that saw the phase complete while another gave up on
+// the abort flag returns false with it. This costs less than one lane polling
+// and broadcasting, then every lane confirming.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned int *err,
+                                          unsigned int site) {
+  const int ok = mbar_wait(bar, parity, abort, err, site) ? 1 : 0;
+  return __all_sync(0xffffffffu, ok) != 0;
+}
+
 // Waits until the counter *ctr (global or shared memory, written by other
 // CTAs or threads with atomics) reaches `target`, sleeping briefly between
 // reads. Gives up after `limit` SM clock cycles, recording the timeout and

@@ -60,15 +60,6 @@ struct TcBars {
   int abort;
 };
 
-__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, unsigned int *err,
-                                          unsigned int site) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, err, site) ? 1 : 0;
-  ok = __shfl_sync(0xffffffffu, ok, 0);
-  if (ok) (void)mbar_try_wait(bar, parity);
-  return ok != 0;
-}
-
 __global__ void split_tf32_kernel(const float4 *x, long long n4, float4 *hi, float4 *lo) {
   pdl_wait();  // the pooled keys come from the previous kernel
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
